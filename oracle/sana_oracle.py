@@ -1,0 +1,399 @@
+"""Float64 CPU oracle for the hybrid linear-softmax attention hot path.
+
+TEST INFRASTRUCTURE ONLY.  This module is imported by ``tests/``, by
+``__graft_entry__.smoke()`` and by the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py``; nothing in the product package imports or executes it,
+and it imports nothing from the product package.  It is plain numpy in
+float64: every function follows one passage of the pages, in the pages' order
+and notation, with no blocking, fusion or reordering beyond what that passage
+states.  A matrix product (``@`` / ``einsum``) is used as a library step.
+
+Sources (cited by page title and section / equation):
+
+* [SV1] "SANA-Video: Efficient Video Generation with Block Linear Diffusion
+  Transformer" (paper notes), sec. 3.2 "Linear Attention with RoPE" (the
+  equation for O_i, and the linear-attention-with-RoPE pseudocode), sec. 3.4
+  "Block Linear Attention with Constant-Memory KV Cache" (the causal equation
+  for O_i, the cumulative-sum state, the complexity table and Algorithm 1),
+  sec. 4.1 (model configuration table).
+* [SV2] "SANA-Video 2.0" (hyper.ai summary of arXiv 2607.21553), Method,
+  "Hybrid attention and block residuals" paragraph and its AttnRes equation
+  h_l = sum_i alpha_{i->l} v_i, alpha = softmax_i((w + phi_tau(t))^T RMSNorm(v_i));
+  the shared-router-query paragraph; Experiments (timestep-free router,
+  block span 8).
+* [SV2-abs] "SANA-Video 2.0" abstract (ai-pulse-lab page): gated linear
+  attention with gated softmax anchors at a 3:1 ratio.
+
+Readings where the pages are silent (each also listed in the design doc):
+
+* 3D RoPE layout: global pair j rotates elements (2j, 2j+1); pairs
+  [0, n_t) use the frame index t, the next n_h the row index h, the last n_w
+  the column index w; within an axis, local pair k has angle
+  pos * theta**(-k / n_axis), theta = 10000; rotation (x, y) ->
+  (x cos - y sin, x sin + y cos).  Positions are integer grid indices from 0,
+  the frame index being absolute (t_offset + local frame).
+* eps = 1e-6 added to the denominator after the dot product ([SV1] sec. 3.2
+  pseudocode names eps without a value).
+* "Gated" = elementwise sigmoid of gate logits G = x W_g on the output.
+* Block-causal: a block sees the whole of itself plus every earlier block
+  (Algorithm 1 updates the cache only after the block is fully denoised);
+  RoPE sits in the numerator exactly as in the bidirectional form.
+* Softmax anchor: the same 3D RoPE applied to raw Q and K (no ReLU),
+  scale 1/sqrt(D), bidirectional.
+* AttnRes: RMSNorm without gain, eps_r = 1e-6, phi_tau(t) = 0; sources in the
+  order [embedding, block summaries..., running partial sum], the partial sum
+  left out while it is empty.
+* Stack: layer l is an anchor iff l % 4 == 3; FFN = W_down SiLU(W_up x) with
+  hidden size ffn_mult * C; sublayer input RMSNorm(h) without gain.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py
+against brute force, closed forms or invariants, except the absolute values
+that only the readings above fix (RoPE layout and frequencies, eps values,
+the anchor's use of RoPE, the FFN form, the empty-partial-sum and last-chunk
+rules): those are "parity unpinned" beyond the readings themselves.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+THETA = 10000.0
+EPS = 1e-6
+RMS_EPS = 1e-6
+
+
+# --------------------------------------------------------------------------
+# feature map and 3D RoPE  ([SV1] sec. 3.2)
+# --------------------------------------------------------------------------
+
+def phi(x):
+    """Kernel feature map phi(x) = ReLU(x) ([SV1] sec. 3.2)."""
+    return np.maximum(x, 0.0)
+
+
+def token_grid(T, H, W, t_offset=0):
+    """Integer (t, h, w) of every token, token n = (t*H + h)*W + w.
+
+    The frame index is absolute: t_offset + local frame."""
+    n = np.arange(T * H * W)
+    t = n // (H * W) + t_offset
+    h = (n // W) % H
+    w = n % W
+    return t, h, w
+
+
+def rope_angles(T, H, W, n_t, n_h, n_w, t_offset=0, theta=THETA):
+    """Angle of every (token, rotary pair): array [N, n_t + n_h + n_w].
+
+    Pair j < n_t follows axis t with local index k = j; the next n_h pairs
+    follow h, the last n_w follow w; angle = pos * theta**(-k / n_axis)."""
+    t, h, w = token_grid(T, H, W, t_offset)
+    cols = []
+    for pos, n_ax in ((t, n_t), (h, n_h), (w, n_w)):
+        k = np.arange(n_ax, dtype=np.float64)
+        freq = theta ** (-k / n_ax) if n_ax > 0 else k
+        cols.append(pos.astype(np.float64)[:, None] * freq[None, :])
+    return np.concatenate(cols, axis=1)
+
+
+def apply_rope(x, angles):
+    """Rotate pairs (2j, 2j+1) of the last axis of x[..., N, D] by angles[N, D/2]."""
+    xe = x[..., 0::2]
+    xo = x[..., 1::2]
+    c = np.cos(angles)
+    s = np.sin(angles)
+    out = np.empty_like(x)
+    out[..., 0::2] = xe * c - xo * s
+    out[..., 1::2] = xe * s + xo * c
+    return out
+
+
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _heads(x, heads):
+    """(B, N, C) -> (B, heads, N, D)."""
+    B, N, C = x.shape
+    return x.reshape(B, N, heads, C // heads).transpose(0, 2, 1, 3)
+
+
+def _merge(x):
+    """(B, heads, N, D) -> (B, N, C)."""
+    B, h, N, D = x.shape
+    return x.transpose(0, 2, 1, 3).reshape(B, N, h * D)
+
+
+# --------------------------------------------------------------------------
+# bidirectional ReLU linear attention with RoPE after the ReLU
+# ([SV1] sec. 3.2, equation for O_i and the pseudocode)
+# --------------------------------------------------------------------------
+
+def linattn_state(k, v, angles, heads):
+    """S = sum_j RoPE(phi(K_j))^T V_j  [B, heads, D, D];  z = sum_j phi(K_j)  [B, heads, D].
+
+    The state of [SV1] sec. 3.4 (cumulative sum of S_j and of phi(K_j)^T)."""
+    kh = _heads(np.asarray(k, np.float64), heads)
+    vh = _heads(np.asarray(v, np.float64), heads)
+    k_phi = phi(kh)
+    k_rope = apply_rope(k_phi, angles)
+    S = np.einsum('bhnd,bhne->bhde', k_rope, vh)
+    z = k_phi.sum(axis=2)
+    return S, z
+
+
+def linattn_apply(q, S, z, angles, heads, gate=None, eps=EPS):
+    """O_i = RoPE(phi(Q_i)) S / (phi(Q_i) . z + eps);  Y = sigmoid(G) * O.
+
+    Numerator with RoPE, denominator without it ([SV1] sec. 3.2)."""
+    qh = _heads(np.asarray(q, np.float64), heads)
+    q_phi = phi(qh)
+    q_rope = apply_rope(q_phi, angles)
+    num = np.einsum('bhnd,bhde->bhne', q_rope, S)
+    den = np.einsum('bhnd,bhd->bhn', q_phi, z)
+    out = _merge(num / (den[..., None] + eps))
+    if gate is not None:
+        out = sigmoid(np.asarray(gate, np.float64)) * out
+    return out
+
+
+def linattn_bidirectional(q, k, v, grid, rope_split, heads, gate=None, eps=EPS,
+                          t_offset=0):
+    """One gated bidirectional linear-attention layer on (B, N, C) inputs.
+
+    grid = (T, H, W); rope_split = (n_t, n_h, n_w).  Returns (Y, S, z)."""
+    T, H, W = grid
+    ang = rope_angles(T, H, W, *rope_split, t_offset=t_offset)
+    S, z = linattn_state(k, v, ang, heads)
+    y = linattn_apply(q, S, z, ang, heads, gate, eps)
+    return y, S, z
+
+
+def linattn_bruteforce(q, k, v, grid, rope_split, heads, gate=None, eps=EPS,
+                       mask=None, t_offset=0):
+    """O(N^2) pairwise form of the same layer (pin P1 / P2).
+
+    O_i = sum_j (RoPE(phi Q_i) . RoPE(phi K_j)) V_j / (sum_j phi Q_i . phi K_j + eps),
+    with an optional boolean mask[i, j] selecting the visible keys."""
+    T, H, W = grid
+    ang = rope_angles(T, H, W, *rope_split, t_offset=t_offset)
+    qh = _heads(np.asarray(q, np.float64), heads)
+    kh = _heads(np.asarray(k, np.float64), heads)
+    vh = _heads(np.asarray(v, np.float64), heads)
+    q_phi, k_phi = phi(qh), phi(kh)
+    q_rope, k_rope = apply_rope(q_phi, ang), apply_rope(k_phi, ang)
+    A_num = np.einsum('bhid,bhjd->bhij', q_rope, k_rope)
+    A_den = np.einsum('bhid,bhjd->bhij', q_phi, k_phi)
+    if mask is not None:
+        A_num = A_num * mask
+        A_den = A_den * mask
+    num = np.einsum('bhij,bhje->bhie', A_num, vh)
+    den = A_den.sum(axis=-1)
+    out = _merge(num / (den[..., None] + eps))
+    if gate is not None:
+        out = sigmoid(np.asarray(gate, np.float64)) * out
+    return out
+
+
+# --------------------------------------------------------------------------
+# block-causal form with a constant-memory state ([SV1] sec. 3.4, Algorithm 1)
+# --------------------------------------------------------------------------
+
+def linattn_block_causal_step(q, k, v, chunk_grid, t_offset, rope_split, heads,
+                              S_prev, z_prev, gate=None, eps=EPS, commit=True):
+    """One block of the block-causal recurrence.
+
+    The block's own (S_c, z_c) are added to the cumulative state; its output
+    uses (S_prev + S_c, z_prev + z_c), i.e. the block sees every earlier block
+    and the whole of itself.  With commit the cumulative state is returned as
+    the new state (the cache update after the last denoising step of
+    Algorithm 1); without it the previous state is returned unchanged.
+    Returns (Y, S_new, z_new)."""
+    T, H, W = chunk_grid
+    ang = rope_angles(T, H, W, *rope_split, t_offset=t_offset)
+    S_c, z_c = linattn_state(k, v, ang, heads)
+    S_tot = np.asarray(S_prev, np.float64) + S_c
+    z_tot = np.asarray(z_prev, np.float64) + z_c
+    y = linattn_apply(q, S_tot, z_tot, ang, heads, gate, eps)
+    if commit:
+        return y, S_tot, z_tot
+    return y, np.array(S_prev, np.float64), np.array(z_prev, np.float64)
+
+
+def linattn_token_recurrence(q, k, v, grid, rope_split, heads, eps=EPS):
+    """Per-token causal recurrence of [SV1] sec. 3.4 (chunk size 1), with RoPE
+    in the numerator: O_i = RoPE(phi Q_i)(sum_{j<i} S_j + S_i) / (phi Q_i (sum_{j<=i} phi K_j) + eps)."""
+    T, H, W = grid
+    ang = rope_angles(T, H, W, *rope_split)
+    qh = _heads(np.asarray(q, np.float64), heads)
+    kh = _heads(np.asarray(k, np.float64), heads)
+    vh = _heads(np.asarray(v, np.float64), heads)
+    B, nh, N, D = qh.shape
+    out = np.zeros_like(vh)
+    S = np.zeros((B, nh, D, vh.shape[-1]))
+    z = np.zeros((B, nh, D))
+    q_phi, k_phi = phi(qh), phi(kh)
+    q_rope, k_rope = apply_rope(q_phi, ang), apply_rope(k_phi, ang)
+    for i in range(N):
+        S = S + np.einsum('bhd,bhe->bhde', k_rope[:, :, i], vh[:, :, i])
+        z = z + k_phi[:, :, i]
+        num = np.einsum('bhd,bhde->bhe', q_rope[:, :, i], S)
+        den = np.einsum('bhd,bhd->bh', q_phi[:, :, i], z)
+        out[:, :, i] = num / (den[..., None] + eps)
+    return _merge(out)
+
+
+# --------------------------------------------------------------------------
+# gated softmax anchor ([SV2-abs]; reading: same 3D RoPE on raw Q, K)
+# --------------------------------------------------------------------------
+
+def softmax_anchor(q, k, v, grid, rope_split, heads, gate=None, scale=None,
+                   rows=None, use_rope=True, t_offset=0):
+    """Y = sigmoid(G) * softmax(RoPE(Q) RoPE(K)^T * scale) V over all keys.
+
+    rows: optional index array of query tokens to evaluate (the others are
+    not computed); the result then has shape (B, len(rows), C).
+    Max-subtracted softmax.  With use_rope=False grid and rope_split are unused."""
+    qh = _heads(np.asarray(q, np.float64), heads)
+    kh = _heads(np.asarray(k, np.float64), heads)
+    vh = _heads(np.asarray(v, np.float64), heads)
+    D = qh.shape[-1]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    if use_rope:
+        ang = rope_angles(*grid, *rope_split, t_offset=t_offset)
+        qh = apply_rope(qh, ang)
+        kh = apply_rope(kh, ang)
+    if rows is not None:
+        qh = qh[:, :, rows]
+    logits = np.einsum('bhid,bhjd->bhij', qh, kh) * scale
+    m = logits.max(axis=-1, keepdims=True)
+    p = np.exp(logits - m)
+    p = p / p.sum(axis=-1, keepdims=True)
+    out = _merge(np.einsum('bhij,bhjd->bhid', p, vh))
+    if gate is not None:
+        g = np.asarray(gate, np.float64)
+        if rows is not None:
+            g = g[:, rows]
+        out = sigmoid(g) * out
+    return out
+
+
+def softmax_naive(q, k, v, scale):
+    """Naive softmax attention without max subtraction, single head (pin P5)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    e = np.exp((q @ k.T) * scale)
+    return (e / e.sum(axis=1, keepdims=True)) @ v
+
+
+# --------------------------------------------------------------------------
+# Block Attention Residuals router ([SV2] AttnRes equation)
+# --------------------------------------------------------------------------
+
+def rmsnorm(x, eps=RMS_EPS):
+    """RMSNorm without gain over the last axis."""
+    x = np.asarray(x, np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+
+
+def attnres_route(sources, w, eps=RMS_EPS):
+    """h = sum_i alpha_i v_i with alpha = softmax_i(w^T RMSNorm(v_i)).
+
+    sources: list of (B, N, C) arrays in the order [embedding, block
+    summaries..., partial sum]; w: (C,) router query (phi_tau(t) = 0).
+    Returns (h, alpha) with alpha of shape (B, N, len(sources))."""
+    V = np.stack([np.asarray(s, np.float64) for s in sources], axis=-2)  # B,N,S,C
+    w = np.asarray(w, np.float64)
+    logits = rmsnorm(V, eps) @ w                                       # B,N,S
+    m = logits.max(axis=-1, keepdims=True)
+    e = np.exp(logits - m)
+    alpha = e / e.sum(axis=-1, keepdims=True)
+    h = np.einsum('bns,bnsc->bnc', alpha, V)
+    return h, alpha
+
+
+# --------------------------------------------------------------------------
+# hybrid stack ([SV2] method paragraph; [SV2-abs] 3:1 interleave)
+# --------------------------------------------------------------------------
+
+def silu(x):
+    return x * sigmoid(x)
+
+
+def is_anchor_layer(l, ratio=4):
+    """Layer l (0-based) is a softmax anchor iff l % ratio == ratio - 1."""
+    return l % ratio == ratio - 1
+
+
+def _attention_sublayer(xh, Wl, grid, rope_split, heads, eps, anchor):
+    C = xh.shape[-1]
+    qkvg = xh @ np.asarray(Wl['qkvg'], np.float64).T
+    q, k, v, g = (qkvg[..., i * C:(i + 1) * C] for i in range(4))
+    if anchor:
+        a = softmax_anchor(q, k, v, grid, rope_split, heads, gate=g)
+    else:
+        a, _, _ = linattn_bidirectional(q, k, v, grid, rope_split, heads, gate=g, eps=eps)
+    return a @ np.asarray(Wl['o'], np.float64).T
+
+
+def _ffn_sublayer(xh, Wl):
+    u = silu(xh @ np.asarray(Wl['up'], np.float64).T)
+    return u @ np.asarray(Wl['down'], np.float64).T
+
+
+def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
+                 block_span=8, ratio=4, use_attnres=True, ffn=True, eps=EPS,
+                 rms_eps=RMS_EPS):
+    """Forward of the hybrid stack.
+
+    With AttnRes: every sublayer reads h = route(V_l) over [embedding,
+    completed block summaries, running partial sum], its output is added to
+    the partial sum, and after every block_span layers the partial sum is
+    frozen as a block summary.  The result is the representation a next layer
+    would read: route(V, w_attn) over the final source set.
+    Without AttnRes: plain pre-norm residual x += sublayer(RMSNorm(x))."""
+    x = np.asarray(x, np.float64)
+    if not use_attnres:
+        for l in range(layers):
+            Wl = weights[l]
+            x = x + _attention_sublayer(rmsnorm(x, rms_eps), Wl, grid, rope_split,
+                                        heads, eps, is_anchor_layer(l, ratio))
+            if ffn:
+                x = x + _ffn_sublayer(rmsnorm(x, rms_eps), Wl)
+        return x
+    summaries = []
+    partial = None
+
+    def sources():
+        return [x] + summaries + ([partial] if partial is not None else [])
+
+    for l in range(layers):
+        Wl = weights[l]
+        h, _ = attnres_route(sources(), w_attn, rms_eps)
+        out = _attention_sublayer(rmsnorm(h, rms_eps), Wl, grid, rope_split, heads,
+                                  eps, is_anchor_layer(l, ratio))
+        partial = out if partial is None else partial + out
+        if ffn:
+            h, _ = attnres_route(sources(), w_ffn, rms_eps)
+            partial = partial + _ffn_sublayer(rmsnorm(h, rms_eps), Wl)
+        if (l + 1) % block_span == 0:
+            summaries.append(partial)
+            partial = None
+    h, _ = attnres_route(sources(), w_attn, rms_eps)
+    return h
+
+
+# --------------------------------------------------------------------------
+# error measure
+# --------------------------------------------------------------------------
+
+def max_rel_err(got, ref):
+    """max_i |got_i - ref_i| / max_i |ref_i| (the parity measure)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    denom = np.max(np.abs(ref))
+    if denom == 0.0:
+        return float(np.max(np.abs(got)))
+    return float(np.max(np.abs(got - ref)) / denom)

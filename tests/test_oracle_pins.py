@@ -1,0 +1,419 @@
+"""Pins of the float64 oracle against brute force, closed forms, library
+routines and invariants (no GPU).  Each pin is chosen so that a plausible
+mistake in the oracle (a dropped term, a wrong sign or index, a transposed
+operand, RoPE in the denominator, a wrong axis split) fails at least one."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sana_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(12345)
+
+
+def rand(*shape):
+    return rng.standard_normal(shape)
+
+
+def rel(a, b):
+    return orc.max_rel_err(a, b)
+
+
+# ---------------------------------------------------------------- RoPE (P3)
+
+def test_rope_angles_hand_worked():
+    g = json.load(open(os.path.join(GOLDEN, "rope_angles_tiny.json")))
+    ang = orc.rope_angles(*g["grid"], *g["split"])
+    for e in g["entries"]:
+        np.testing.assert_allclose(ang[e["token"]], e["angles"], rtol=1e-12, atol=1e-15)
+        T, H, W = g["grid"]
+        t, h, w = orc.token_grid(T, H, W)
+        assert [t[e["token"]], h[e["token"]], w[e["token"]]] == e["thw"]
+
+
+def test_rope_single_pair_closed_form():
+    # D = 2: (x, y) rotated by a -> (x cos a - y sin a, x sin a + y cos a)
+    x, y, a = 0.7, -1.3, 0.9
+    out = orc.apply_rope(np.array([[x, y]]), np.array([[a]]))
+    exp = [x * math.cos(a) - y * math.sin(a), x * math.sin(a) + y * math.cos(a)]
+    np.testing.assert_allclose(out[0], exp, rtol=1e-15)
+
+
+def test_rope_preserves_pair_norms():
+    x = rand(3, 40, 16)
+    ang = rand(40, 8) * 5
+    r = orc.apply_rope(x, ang)
+    np.testing.assert_allclose(np.hypot(r[..., 0::2], r[..., 1::2]),
+                               np.hypot(x[..., 0::2], x[..., 1::2]), rtol=1e-13)
+
+
+def test_rope_offset_absolute_frames():
+    a0 = orc.rope_angles(3, 2, 2, 2, 1, 1, t_offset=5)
+    a1 = orc.rope_angles(8, 2, 2, 2, 1, 1)[5 * 4:]
+    np.testing.assert_allclose(a0, a1, rtol=0, atol=0)
+
+
+# ------------------------------------------------- bidirectional linear attention
+
+def _lin_inputs(B, N, heads, D, gate=True):
+    C = heads * D
+    return (rand(B, N, C), rand(B, N, C), rand(B, N, C),
+            rand(B, N, C) if gate else None)
+
+
+@pytest.mark.parametrize("grid,split,heads,D", [
+    ((2, 4, 4), (2, 3, 3), 2, 16),      # the tiny workload
+    ((3, 5, 7), (2, 3, 3), 1, 16),      # N = 105, ragged against any tile size
+    ((5, 7, 8), (1, 1, 2), 3, 8),       # N = 280
+    ((1, 1, 1), (0, 0, 4), 2, 8),       # a single token
+])
+def test_factorised_equals_bruteforce(grid, split, heads, D):
+    """P1: the associativity of the linear form (sec. 3.2 pseudocode)."""
+    N = grid[0] * grid[1] * grid[2]
+    q, k, v, g = _lin_inputs(2, N, heads, D)
+    y, S, z = orc.linattn_bidirectional(q, k, v, grid, split, heads, gate=g)
+    yb = orc.linattn_bruteforce(q, k, v, grid, split, heads, gate=g)
+    assert rel(y, yb) < 1e-12
+
+
+def test_linear_attention_d2_worked_example():
+    """A hand-worked D = 2 example: one head, tokens at w = 0 and w = 1
+    (angle 0 and 1 rad).  q0=(1,0), q1=(.5,2), k0=(1,1), k1=(2,-1),
+    v0=(1,2), v1=(3,-1).  phi(k1) = (2,0), so
+    S = [[1 + 6 cos1, 2 - 2 cos1], [1 + 6 sin1, 2 - 2 sin1]], z = (3, 1).
+    Token 0: numerator = row 0 of S, denominator 3.
+    Token 1: RoPE(phi q1) = (.5 cos1 - 2 sin1, .5 sin1 + 2 cos1), denominator
+    .5*3 + 2*1 = 3.5."""
+    c, s = math.cos(1.0), math.sin(1.0)
+    S = np.array([[1 + 6 * c, 2 - 2 * c], [1 + 6 * s, 2 - 2 * s]])
+    eps = orc.EPS
+    o0 = S[0] / (3 + eps)
+    qr = np.array([0.5 * c - 2 * s, 0.5 * s + 2 * c])
+    o1 = (qr @ S) / (3.5 + eps)
+    q = np.array([[[1, 0], [0.5, 2]]], float)
+    k = np.array([[[1, 1], [2, -1]]], float)
+    v = np.array([[[1, 2], [3, -1]]], float)
+    y, S_o, z_o = orc.linattn_bidirectional(q, k, v, (1, 1, 2), (0, 0, 1), 1)
+    np.testing.assert_allclose(S_o[0, 0], S, rtol=1e-14)
+    np.testing.assert_allclose(z_o[0, 0], [3, 1], rtol=1e-15)
+    np.testing.assert_allclose(y[0], np.stack([o0, o1]), rtol=1e-13)
+
+
+def test_positions_zero_reduce_to_plain_relu_linear_attention():
+    """P3/P4: with every angle 0 RoPE is the identity; with V = c the output
+    is c * d / (d + eps) with d = phi(Q) . z."""
+    N, D = 24, 8
+    q, k, _, _ = _lin_inputs(1, N, 1, D, gate=False)
+    # a grid of a single position on every axis used: all angles zero
+    ang0 = np.zeros((N, D // 2))
+    S, z = orc.linattn_state(k, np.ones((1, N, D)) * 1.5, ang0, 1)
+    y = orc.linattn_apply(q, S, z, ang0, 1)
+    d = np.maximum(q, 0) @ np.maximum(k, 0)[0].sum(0)
+    np.testing.assert_allclose(y[0], (1.5 * d / (d + orc.EPS))[0][:, None] * np.ones(D),
+                               rtol=1e-12)
+    # and the general no-RoPE case equals plain ReLU linear attention
+    v = rand(1, N, D)
+    S, z = orc.linattn_state(k, v, ang0, 1)
+    y = orc.linattn_apply(q, S, z, ang0, 1)
+    qp, kp = np.maximum(q[0], 0), np.maximum(k[0], 0)
+    plain = (qp @ kp.T @ v[0]) / ((qp @ kp.T).sum(1, keepdims=True) + orc.EPS)
+    assert rel(y[0], plain) < 1e-12
+
+
+def test_denominator_carries_no_rope():
+    """The denominator is phi(Q).sum phi(K) without rotation: with V = 1 and
+    angles != 0 the output differs from the rotated-denominator variant."""
+    grid, split = (2, 3, 3), (1, 1, 2)
+    N, D = 18, 8
+    q, k, _, _ = _lin_inputs(1, N, 1, D, gate=False)
+    ang = orc.rope_angles(*grid, *split)
+    S, z = orc.linattn_state(k, rand(1, N, D), ang, 1)
+    qp = np.maximum(q[0], 0)
+    den_norope = qp @ np.maximum(k[0], 0).sum(0)
+    y = orc.linattn_apply(q, S, z, ang, 1)
+    num = orc.apply_rope(qp, ang) @ S[0, 0]
+    np.testing.assert_allclose(y[0], num / (den_norope[:, None] + orc.EPS), rtol=1e-12)
+
+
+def test_relative_position_shift_invariance():
+    """P3: shifting every frame index leaves the bidirectional output unchanged."""
+    grid, split = (3, 3, 4), (2, 1, 1)
+    N = 36
+    q, k, v, g = _lin_inputs(1, N, 2, 8)
+    y0, _, _ = orc.linattn_bidirectional(q, k, v, grid, split, 2, gate=g)
+    y1, _, _ = orc.linattn_bidirectional(q, k, v, grid, split, 2, gate=g, t_offset=17)
+    assert rel(y1, y0) < 1e-12
+
+
+def test_gate_limits():
+    """P7: gate logits -> +inf give the ungated output, -> -inf give 0."""
+    grid, split = (2, 2, 2), (1, 1, 2)
+    q, k, v, _ = _lin_inputs(1, 8, 1, 8, gate=False)
+    y, _, _ = orc.linattn_bidirectional(q, k, v, grid, split, 1)
+    yp, _, _ = orc.linattn_bidirectional(q, k, v, grid, split, 1, gate=np.full(q.shape, 60.0))
+    ym, _, _ = orc.linattn_bidirectional(q, k, v, grid, split, 1, gate=np.full(q.shape, -60.0))
+    assert rel(yp, y) < 1e-15
+    assert np.max(np.abs(ym)) <= 1e-25 * np.max(np.abs(y))
+
+
+def test_state_size_independent_of_n():
+    """P8: the state is D x D plus D per head whatever N is (sec. 3.4 table)."""
+    for T in (1, 4, 9):
+        grid = (T, 2, 2)
+        N = 4 * T
+        _, k, v, _ = _lin_inputs(1, N, 3, 8, gate=False)
+        S, z = orc.linattn_state(k, v, orc.rope_angles(*grid, 1, 1, 2), 3)
+        assert S.shape == (1, 3, 8, 8) and z.shape == (1, 3, 8)
+
+
+# ------------------------------------------------------------- block-causal (P2)
+
+def _frame_mask(grid, chunk_sizes):
+    T, H, W = grid
+    frame_chunk = np.concatenate([[c] * f for c, f in enumerate(chunk_sizes)])
+    tok_chunk = np.repeat(frame_chunk, H * W)
+    return tok_chunk[None, :] <= tok_chunk[:, None]
+
+
+def _run_chunks(q, k, v, g, grid, split, heads, chunk_sizes, S0=None, z0=None, eps=orc.EPS):
+    T, H, W = grid
+    B, N, C = q.shape
+    D = C // heads
+    S = np.zeros((B, heads, D, D)) if S0 is None else S0
+    z = np.zeros((B, heads, D)) if z0 is None else z0
+    ys, states = [], []
+    t0 = 0
+    for f in chunk_sizes:
+        sl = slice(t0 * H * W, (t0 + f) * H * W)
+        y, S, z = orc.linattn_block_causal_step(
+            q[:, sl], k[:, sl], v[:, sl], (f, H, W), t0, split, heads, S, z,
+            gate=None if g is None else g[:, sl], eps=eps)
+        ys.append(y)
+        states.append((S.copy(), z.copy()))
+        t0 += f
+    return np.concatenate(ys, axis=1), states
+
+
+@pytest.mark.parametrize("chunks", [[1] * 6, [2, 2, 2], [3, 3], [5, 1], [1, 2, 3], [6]])
+def test_chunked_equals_masked_bruteforce(chunks):
+    grid, split, heads = (6, 2, 3), (2, 1, 1), 2
+    N = 36
+    q, k, v, g = _lin_inputs(1, N, heads, 8)
+    y, _ = _run_chunks(q, k, v, g, grid, split, heads, chunks)
+    yb = orc.linattn_bruteforce(q, k, v, grid, split, heads, gate=g,
+                                mask=_frame_mask(grid, chunks))
+    assert rel(y, yb) < 1e-12
+
+
+def test_token_recurrence_equals_prefix_recomputation():
+    """Chunk size 1 token: the sec. 3.4 recurrence = brute force with j <= i."""
+    grid, split, heads = (2, 3, 4), (2, 1, 1), 2
+    N = 24
+    q, k, v, _ = _lin_inputs(1, N, heads, 8, gate=False)
+    y = orc.linattn_token_recurrence(q, k, v, grid, split, heads)
+    mask = np.tril(np.ones((N, N), bool))
+    yb = orc.linattn_bruteforce(q, k, v, grid, split, heads, mask=mask)
+    assert rel(y, yb) < 1e-12
+
+
+def test_state_independent_of_chunking_and_full_chunk_is_bidirectional():
+    grid, split, heads = (6, 2, 2), (2, 1, 1), 2
+    q, k, v, g = _lin_inputs(2, 24, heads, 8)
+    _, st_a = _run_chunks(q, k, v, g, grid, split, heads, [1, 2, 3])
+    _, st_b = _run_chunks(q, k, v, g, grid, split, heads, [3, 3])
+    _, st_c = _run_chunks(q, k, v, g, grid, split, heads, [6])
+    # state after the first 3 frames
+    assert rel(st_a[1][0], st_b[0][0]) < 1e-13 and rel(st_a[1][1], st_b[0][1]) < 1e-13
+    for st in (st_a[-1], st_b[-1]):
+        assert rel(st[0], st_c[-1][0]) < 1e-13 and rel(st[1], st_c[-1][1]) < 1e-13
+    y_full, _ = _run_chunks(q, k, v, g, grid, split, heads, [6])
+    y_bi, S, z = orc.linattn_bidirectional(q, k, v, grid, split, heads, gate=g)
+    assert rel(y_full, y_bi) < 1e-13
+    assert rel(st_c[-1][0], S) < 1e-13 and rel(st_c[-1][1], z) < 1e-13
+
+
+def test_commit_flag_and_state_save_restore():
+    grid, split, heads = (4, 2, 2), (2, 1, 1), 1
+    q, k, v, _ = _lin_inputs(1, 16, heads, 8, gate=False)
+    H, W = 2, 2
+    S0 = np.zeros((1, 1, 8, 8))
+    z0 = np.zeros((1, 1, 8))
+    y1, S1, z1 = orc.linattn_block_causal_step(q[:, :8], k[:, :8], v[:, :8], (2, H, W), 0,
+                                               split, heads, S0, z0)
+    # a non-committing step leaves the state untouched but sees itself
+    y_nc, S_nc, z_nc = orc.linattn_block_causal_step(q[:, 8:], k[:, 8:], v[:, 8:], (2, H, W), 2,
+                                                     split, heads, S1, z1, commit=False)
+    assert np.array_equal(S_nc, S1) and np.array_equal(z_nc, z1)
+    # save / restore through a byte round trip is exact
+    S_r = np.frombuffer(S1.tobytes()).reshape(S1.shape)
+    z_r = np.frombuffer(z1.tobytes()).reshape(z1.shape)
+    y2, _, _ = orc.linattn_block_causal_step(q[:, 8:], k[:, 8:], v[:, 8:], (2, H, W), 2,
+                                             split, heads, S_r, z_r)
+    assert np.array_equal(y2, y_nc)
+
+
+# ------------------------------------------------------------------ anchor (P5)
+
+def test_anchor_equals_naive_softmax_and_library_sdpa():
+    N, D, heads = 40, 8, 2
+    q, k, v = rand(1, N, heads * D) * 0.3, rand(1, N, heads * D) * 0.3, rand(1, N, heads * D)
+    y = orc.softmax_anchor(q, k, v, None, None, heads, use_rope=False)
+    for h in range(heads):
+        sl = slice(h * D, (h + 1) * D)
+        yn = orc.softmax_naive(q[0, :, sl], k[0, :, sl], v[0, :, sl], D ** -0.5)
+        assert rel(y[0, :, sl], yn) < 1e-13
+        ys = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[0, :, sl])[None], torch.from_numpy(k[0, :, sl])[None],
+            torch.from_numpy(v[0, :, sl])[None]).numpy()[0]
+        assert rel(y[0, :, sl], ys) < 1e-12
+
+
+def test_anchor_with_rope_equals_sdpa_on_rotated_inputs():
+    grid, split, heads, D = (2, 3, 4), (1, 1, 2), 2, 8
+    N = 24
+    q, k, v = rand(1, N, heads * D), rand(1, N, heads * D), rand(1, N, heads * D)
+    g = rand(1, N, heads * D)
+    y = orc.softmax_anchor(q, k, v, grid, split, heads, gate=g)
+    ang = orc.rope_angles(*grid, *split)
+    for h in range(heads):
+        sl = slice(h * D, (h + 1) * D)
+        qr = torch.from_numpy(orc.apply_rope(q[0, :, sl], ang))[None]
+        kr = torch.from_numpy(orc.apply_rope(k[0, :, sl], ang))[None]
+        ys = torch.nn.functional.scaled_dot_product_attention(
+            qr, kr, torch.from_numpy(v[0, :, sl])[None]).numpy()[0]
+        assert rel(y[0, :, sl], ys / (1 + np.exp(-g[0, :, sl]))) < 1e-12
+    # sampled rows equal the full evaluation
+    rows = np.array([0, 5, 23])
+    assert rel(orc.softmax_anchor(q, k, v, grid, split, heads, gate=g, rows=rows),
+               y[:, rows]) < 1e-15
+
+
+def test_anchor_special_cases():
+    grid, split, heads, D = (1, 2, 5), (0, 2, 2), 1, 8
+    N = 10
+    q, k = rand(1, N, D), rand(1, N, D)
+    v = np.full((1, N, D), 2.5)
+    np.testing.assert_allclose(orc.softmax_anchor(q, k, v, grid, split, heads), v, rtol=1e-14)
+    # a single key: every query returns that key's value
+    y1 = orc.softmax_anchor(q[:, :1], k[:, :1], rand(1, 1, D), (1, 1, 1), split, heads)
+    assert y1.shape == (1, 1, D)
+    # a constant added to all logits of a row changes nothing (K + c shifts each
+    # row of Q K^T by q_i . c when RoPE is off)
+    v = rand(1, N, D)
+    y = orc.softmax_anchor(q, k, v, None, None, heads, use_rope=False)
+    y2 = orc.softmax_anchor(q, k + rand(1, 1, D), v, None, None, heads, use_rope=False)
+    assert rel(y2, y) < 1e-12
+    # relative RoPE: a frame shift leaves the anchor unchanged
+    grid2 = (3, 2, 2)
+    q, k, v = rand(1, 12, D), rand(1, 12, D), rand(1, 12, D)
+    a = orc.softmax_anchor(q, k, v, grid2, (2, 1, 1), 1)
+    b = orc.softmax_anchor(q, k, v, grid2, (2, 1, 1), 1, t_offset=11)
+    assert rel(a, b) < 1e-12
+
+
+# ------------------------------------------------------------------ AttnRes (P6)
+
+def test_attnres_two_source_closed_form():
+    """C = 4, v1 = a e1 (a > 0), v2 = 0.  RMSNorm(v1) = a e1 / sqrt(a^2/4 + eps),
+    RMSNorm(0) = 0.  With w = (L, 0, 0, 0) the logits are
+    L * a / sqrt(a^2/4 + eps) and 0, so alpha = softmax of those and
+    h = alpha_1 v1."""
+    a, L = 3.0, 0.4
+    v1 = np.zeros((1, 1, 4)); v1[..., 0] = a
+    v2 = np.zeros((1, 1, 4))
+    w = np.array([L, 0, 0, 0])
+    l1 = L * a / math.sqrt(a * a / 4 + orc.RMS_EPS)
+    a1 = math.exp(l1) / (math.exp(l1) + 1.0)
+    h, alpha = orc.attnres_route([v1, v2], w)
+    np.testing.assert_allclose(alpha[0, 0], [a1, 1 - a1], rtol=1e-14)
+    np.testing.assert_allclose(h[0, 0], [a1 * a, 0, 0, 0], rtol=1e-14)
+
+
+def test_attnres_invariants():
+    B, N, C = 2, 7, 32
+    srcs = [rand(B, N, C) for _ in range(4)]
+    w = rand(C) / math.sqrt(C)
+    h, alpha = orc.attnres_route(srcs, w)
+    np.testing.assert_allclose(alpha.sum(-1), 1.0, rtol=1e-14)
+    # one source: h = v exactly
+    h1, a1 = orc.attnres_route(srcs[:1], w)
+    assert np.array_equal(h1, srcs[0]) and np.all(a1 == 1.0)
+    # permuting the sources permutes alpha and leaves h unchanged
+    perm = [2, 0, 3, 1]
+    hp, ap = orc.attnres_route([srcs[i] for i in perm], w)
+    assert rel(hp, h) < 1e-14
+    np.testing.assert_allclose(ap, alpha[..., perm], rtol=1e-13)
+    # scaling a source by s > 0 leaves its logit unchanged (up to eps)
+    hs, as_ = orc.attnres_route([srcs[0] * 7.0] + srcs[1:], w)
+    np.testing.assert_allclose(as_, alpha, rtol=1e-5)
+    # w = 0: the mean of the sources
+    h0, _ = orc.attnres_route(srcs, np.zeros(C))
+    np.testing.assert_allclose(h0, np.mean(srcs, axis=0), rtol=1e-13)
+
+
+def test_rmsnorm_closed_form():
+    x = np.full((1, 8), -2.0)
+    np.testing.assert_allclose(orc.rmsnorm(x), -2.0 / math.sqrt(4.0 + orc.RMS_EPS), rtol=1e-15)
+
+
+# -------------------------------------------------------------------- stack
+
+def test_schedule_matches_page_constants():
+    c = json.load(open(os.path.join(GOLDEN, "page_constants.json")))
+    lin, soft = c["linear_to_softmax_ratio"]
+    ratio = lin + soft
+    anchors = [l for l in range(16) if orc.is_anchor_layer(l, ratio)]
+    assert anchors == [3, 7, 11, 15]
+    assert len(anchors) / 16 == c["softmax_fraction"]
+    assert c["attnres_block_span"] == 8 and c["shared_router_queries"] == 2
+    v1 = c["v1_model"]
+    assert v1["width"] == v1["heads"] * v1["head_dim"] and v1["ffn"] == 3 * v1["width"]
+
+
+def _zero_stack_weights(layers, C, F):
+    return [dict(qkvg=rand(4 * C, C) / math.sqrt(C), o=np.zeros((C, C)),
+                 up=rand(F, C) / math.sqrt(C), down=np.zeros((C, F))) for _ in range(layers)]
+
+
+@pytest.mark.parametrize("layers,span", [(16, 8), (5, 2), (3, 8)])
+def test_stack_block_bookkeeping_closed_form(layers, span):
+    """With W_o = W_down = 0 every sublayer output is 0, so the partial sum and
+    every block summary are 0 (RMSNorm(0) = 0, logit 0).  The output is
+    route([x, 0 * nsum]) = x * e^l / (e^l + nsum) with l = w . RMSNorm(x) and
+    nsum = layers // span completed summaries (the partial sum is empty after a
+    completed block and 0 otherwise, adding one more zero source)."""
+    grid, split, heads, D = (2, 2, 2), (1, 1, 2), 2, 8
+    C, N = heads * D, 8
+    x = rand(1, N, C)
+    w_attn, w_ffn = rand(C) / 4, rand(C) / 4
+    ws = _zero_stack_weights(layers, C, 3 * C)
+    out = orc.hybrid_stack(x, ws, w_attn, w_ffn, grid, split, heads, layers, block_span=span)
+    nzero = layers // span + (1 if layers % span else 0)
+    lx = orc.rmsnorm(x) @ w_attn
+    exp = x * (np.exp(lx) / (np.exp(lx) + nzero))[..., None]
+    assert rel(out, exp) < 1e-13
+
+
+def test_stack_without_attnres_is_residual_composition():
+    grid, split, heads, D = (2, 2, 2), (1, 1, 2), 2, 8
+    C, N = heads * D, 8
+    x = rand(1, N, C)
+    ws = [dict(qkvg=rand(4 * C, C) / 4, o=rand(C, C) / 4) for _ in range(4)]
+    out = orc.hybrid_stack(x, ws, None, None, grid, split, heads, 4, use_attnres=False, ffn=False)
+    ref = x.copy()
+    for l in range(4):
+        xh = ref / np.sqrt(np.mean(ref ** 2, -1, keepdims=True) + orc.RMS_EPS)
+        qkvg = xh @ ws[l]["qkvg"].T
+        q, k, v, g = (qkvg[..., i * C:(i + 1) * C] for i in range(4))
+        if l == 3:
+            a = orc.softmax_anchor(q, k, v, grid, split, heads, gate=g)
+        else:
+            a = orc.linattn_bruteforce(q, k, v, grid, split, heads, gate=g)
+        ref = ref + a @ ws[l]["o"].T
+    assert rel(out, ref) < 1e-12
