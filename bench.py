@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the gated ReLU-RoPE linear-attention layer at the 720p/5s
+latent shape (B=1, T=21, H=45, W=80 -> N=75,600 tokens, 24 heads, D=128,
+bf16, sigmoid output gate) on B200, through libsana's C ABI.
+
+One step = one sana_linattn_fwd call: ReLU + RoPE of K, the N-axis state
+reduction S = sum RoPE(phi K)^T V and z = sum phi K, the fixed-order combine,
+ReLU + RoPE of Q, the numerator Q'S, the RoPE-free denominator, and the
+sigmoid gate.  Inputs (4 x 464.5 MB) exceed the 126 MB L2, so no flush is
+needed between steps.
+
+`value` is whole-job tokens/s (all ranks; each rank runs its own layer, weak
+scaling), device-timed with CUDA events, max over ranks.  Rank 0 prints one
+JSON line.  `--impl reference` times the float64 CPU oracle instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sana_inputs as si  # noqa: E402
+
+METRIC = "linear-attn tokens/s and TFLOP/s per layer @720p/5s bf16; % of roofline"
+WL = si.P720
+TENSOR_BYTES = WL.B * WL.N * WL.C * 2                  # one (B, N, C) bf16 tensor
+LAYER_BYTES = 5 * TENSOR_BYTES                         # Q, K, V, G read; Y written
+APPLY_BYTES = 3 * TENSOR_BYTES                         # output kernel: Q, G read; Y written
+LAYER_FLOPS = 4 * WL.B * WL.N * WL.heads * WL.D ** 2   # K'^T V and Q' S
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("linattn_tc.cu", "sana_common.cuh", "rope_dev.cuh"):
+        h.update(open(os.path.join(ROOT, "softmax_attention_sana_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the output kernel from the committed ncu summary,
+    if it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "linattn_out_kernel_720p.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_h = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", txt)
+    m_t = re.search(r"dram bytes per launch:\s*`?([0-9.eE+]+)", txt)
+    if not (m_h and m_t) or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_loop(fn, steps):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps  # ms
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_inputs(heads, cpu_tensors=None):
+    """float64 copies of the first `heads` heads of the 720p layer's inputs."""
+    if heads not in _ORACLE_INPUTS:
+        ts = cpu_tensors if cpu_tensors is not None else si.qkvg(WL)
+        cols = slice(0, heads * WL.D)
+        _ORACLE_INPUTS[heads] = tuple(si.as_f64(t[..., cols]) for t in ts)
+    return _ORACLE_INPUTS[heads]
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # pragma: no cover
+        return os.cpu_count()
+
+
+def oracle_sample(heads, n_tok, cpu_tensors=None):
+    """Time the float64 oracle on `heads` heads and the first `n_tok` tokens of
+    the 720p layer (state over those tokens, then their outputs).  The oracle's
+    work is linear in heads x tokens, so the time scales to a whole layer by
+    (24 / heads) x (N / n_tok).  Returns (tokens/s of a layer, seconds, text)."""
+    from oracle import sana_oracle as orc
+    q, k, v, g = (t[:, :n_tok] for t in oracle_inputs(heads, cpu_tensors))
+    t0 = time.perf_counter()
+    ang = orc.rope_angles(WL.T, WL.H, WL.W, *WL.rope_split)[:n_tok]
+    S, z = orc.linattn_state(k, v, ang, heads)
+    orc.linattn_apply(q, S, z, ang, heads, gate=g)
+    dt = time.perf_counter() - t0
+    scale = (WL.heads / heads) * (WL.N / n_tok)
+    desc = (f"oracle (numpy float64) on {heads} of {WL.heads} heads x {n_tok} of {WL.N} tokens "
+            f"of the 720p layer, time scaled x{scale:.2f} to a whole layer")
+    return WL.B * WL.N / (dt * scale), dt, desc
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    # calibrate the per-(head, token) cost, then size each step's sample so the
+    # whole --steps/--warmup run takes about args.ref_budget seconds
+    _, dt, _ = oracle_sample(1, 4096)
+    _, dt, _ = oracle_sample(1, 4096)
+    per_tok = dt / 4096
+    budget = max(0.02, min(5.0, args.ref_budget / (args.steps + args.warmup)))
+    n_tok = int(min(WL.N, max(512, budget / per_tok)))
+    for _ in range(args.warmup):
+        oracle_sample(1, n_tok)
+    vals = []
+    desc = ""
+    for _ in range(args.steps):
+        v, _, desc = oracle_sample(1, n_tok)
+        vals.append(v)
+    value = float(np.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * WL.B * WL.N / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc + " (median over steps)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config():
+    return {"workload": "720p/5s gated linear-attention layer", "B": WL.B, "T": WL.T, "H": WL.H,
+            "W": WL.W, "N": WL.N, "heads": WL.heads, "head_dim": WL.D, "gate": "sigmoid",
+            "rope_split": list(WL.rope_split),
+            "l2": "no flush: 4 inputs x 464.5 MB per step exceed the 126 MB L2"}
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def components(sana, args):
+    """Other rows of the hot path, each timed on its own with CUDA events."""
+    out = {}
+    # 480p layer
+    wl = si.P480
+    q, k, v, g = (t.cuda() for t in si.qkvg(wl))
+    rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
+    ws = torch.empty(sana.linattn_workspace_size(wl.B, (wl.T, wl.H, wl.W), wl.heads, wl.D, 1),
+                     dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(q)
+    f = lambda: sana.linattn_fwd(q, k, v, g, rope, (wl.T, wl.H, wl.W), wl.heads, out=y, ws=ws)
+    for _ in range(5):
+        f()
+    ms = time_loop(f, 50)
+    out["linattn_480p"] = {"ms": ms, "tokens_per_s": wl.N / (ms / 1e3),
+                           "GB_per_s": 5 * wl.N * wl.C * 2 / (ms / 1e3) / 1e9}
+    del q, k, v, g, y
+    # block-causal chunk step (720p/60s chunk: 3 frames, 10,800 tokens, state carried)
+    wl = si.LONG
+    q, k, v = (t.cuda() for t in si.causal_chunk(wl, 0, 3))
+    rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
+    S = torch.zeros(1, wl.heads, wl.D, wl.D, device="cuda")
+    z = torch.zeros(1, wl.heads, wl.D, device="cuda")
+    ws = torch.empty(sana.linattn_workspace_size(1, (3, wl.H, wl.W), wl.heads, wl.D, 1),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(q)
+    f = lambda: sana.linattn_block_causal_step(q, k, v, None, rope, (3, wl.H, wl.W), 3, wl.heads,
+                                               S, z, commit=True, out=y, ws=ws)
+    for _ in range(5):
+        f()
+    # L2 flush between timed chunk steps (inputs are smaller than L2)
+    s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot = 0.0
+    for _ in range(20):
+        flush.zero_()
+        torch.cuda.synchronize()
+        s_ev.record()
+        f()
+        e_ev.record()
+        torch.cuda.synchronize()
+        tot += s_ev.elapsed_time(e_ev)
+    ms = tot / 20
+    nb = 4 * 10800 * wl.C * 2 + 2 * 4 * wl.heads * (wl.D * wl.D + wl.D)
+    out["causal_chunk_720p60s"] = {"ms": ms, "tokens_per_s": 10800 / (ms / 1e3),
+                                   "GB_per_s": nb / (ms / 1e3) / 1e9, "l2": "flushed (256 MB) per step"}
+    del q, k, v, y, flush
+    # AttnRes route over 3 sources at 720p/5s
+    srcs = [t.cuda() for t in si.attnres_sources(5, 3, 1, si.P720.N, si.P720.C)]
+    w_attn, _ = (t.cuda() for t in si.router_queries(5, si.P720.C))
+    h = torch.empty_like(srcs[0])
+    f = lambda: sana.attnres_route(srcs, w_attn, out=h)
+    for _ in range(3):
+        f()
+    ms = time_loop(f, 20)
+    out["attnres_route_720p_3src"] = {"ms": ms, "GB_per_s": 4 * TENSOR_BYTES / (ms / 1e3) / 1e9}
+    del srcs, h
+    # softmax anchor at 720p/5s
+    try:
+        q, k, v, g = (t.cuda() for t in si.qkvg(WL))
+        rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
+        ws = torch.empty(int(4 * TENSOR_BYTES // 2 + (1 << 20)), dtype=torch.uint8, device="cuda")
+        y = torch.empty_like(q)
+        f = lambda: sana.softmax_anchor_fwd(q, k, v, g, rope, (WL.T, WL.H, WL.W), WL.heads, out=y,
+                                            ws=ws)
+        f()
+        ms = time_loop(f, 3)
+        flops = 4 * WL.N * WL.N * WL.heads * WL.D
+        out["softmax_anchor_720p"] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}
+    except Exception as e:  # not built yet
+        out["softmax_anchor_720p"] = {"unavailable": str(e)[:200]}
+    return out
+
+
+def run_ours(args, world, rank, local):
+    import softmax_attention_sana_b200 as sana
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    grid = (WL.T, WL.H, WL.W)
+    cpu_inputs = si.qkvg(WL)
+    q, k, v, g = (t.to(dev) for t in cpu_inputs)
+    rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
+    ws = torch.empty(sana.linattn_workspace_size(WL.B, grid, WL.heads, WL.D, 1), dtype=torch.uint8,
+                     device=dev)
+    y = torch.empty_like(q)
+    step = lambda: sana.linattn_fwd(q, k, v, g, rope, grid, WL.heads, out=y, ws=ws)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    sana.sync_status()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    ms = time_loop(step, args.steps)
+    barrier(world)
+    clocks.mark("t1")
+    sana.sync_status()
+    ms = max_over_ranks(ms, world)
+    clk = clocks.stop()
+
+    # dominant kernel: the output pass (Q, G read, Y written), one launch per call
+    S, z = sana.linattn_state(k, v, rope, grid, WL.heads)
+    apply = lambda: sana.linattn_apply(q, g, rope, grid, WL.heads, S, z, out=y)
+    for _ in range(3):
+        apply()
+    ms_apply = time_loop(apply, max(10, args.steps))
+    st_ws = torch.empty(max(256, sana._lib.linattn_state_workspace_size(WL.B, grid, WL.heads, WL.D, 1)),
+                        dtype=torch.uint8, device=dev)
+    state = lambda: sana.linattn_state(k, v, rope, grid, WL.heads, S=S, z=z, ws=st_ws)
+    for _ in range(3):
+        state()
+    ms_state = time_loop(state, max(10, args.steps))
+    sana.sync_status()
+
+    # end to end through the C ABI with pinned host buffers
+    hq, hk, hv, hg = (t.cpu().pin_memory() for t in (q, k, v, g))
+    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    dq, dk, dv, dg = (torch.empty_like(t) for t in (q, k, v, g))
+
+    def e2e_step():
+        for d, h in ((dq, hq), (dk, hk), (dv, hv), (dg, hg)):
+            d.copy_(h, non_blocking=True)
+        sana.linattn_fwd(dq, dk, dv, dg, rope, grid, WL.heads, out=y, ws=ws)
+        hy.copy_(y, non_blocking=True)
+
+    e2e_step()
+    ms_e2e = max_over_ranks(time_loop(e2e_step, args.e2e_steps), world)
+    sana.sync_status()
+
+    comp = components(sana, args) if (world == 1 and args.components == "all") else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, dt, desc = oracle_sample(args.ref_heads, WL.N, cpu_inputs)
+        cpu = {"value": v_cpu, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f" ({dt:.1f} s of CPU time)"}
+
+    if rank != 0:
+        return
+    hbm, peak_kind = peaks()
+    ach_apply = APPLY_BYTES / (ms_apply / 1e3) / 1e9
+    ach_layer = LAYER_BYTES / (ms / 1e3) / 1e9
+    tokens = world * WL.B * WL.N
+    line = {
+        "metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(),
+        "tflops_per_layer": LAYER_FLOPS / (ms / 1e3) / 1e12,
+        "roofline": {"bound": "hbm", "kernel": "linattn_out_kernel (output pass: Q, G read, Y written)",
+                     "achieved": ach_apply, "peak": hbm, "unit": "GB/s", "frac": ach_apply / hbm,
+                     "peak_kind": peak_kind, "traffic": recorded_traffic(),
+                     "algorithmic_bytes_per_launch": APPLY_BYTES, "ms_per_launch": ms_apply},
+        "layer_roofline": {"bound": "hbm", "achieved": ach_layer, "peak": hbm, "unit": "GB/s",
+                           "frac": ach_layer / hbm, "algorithmic_bytes": LAYER_BYTES,
+                           "state_phase_ms": ms_state, "apply_phase_ms": ms_apply},
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 * TENSOR_BYTES, "d2h_bytes_per_step": TENSOR_BYTES,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if comp is not None:
+        line["components"] = comp
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--components", choices=["all", "none"], default="all")
+    ap.add_argument("--ref-heads", type=int, default=12,
+                    help="heads of the 720p layer in the cpu_baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="seconds the --impl reference run aims to take")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,253 @@
+/*
+ * libsana — C ABI of the SANA-Video 2.0 hybrid linear-softmax attention hot path
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Operations (cited by page title and section / equation):
+ *   [SV1]  "SANA-Video: Efficient Video Generation with Block Linear Diffusion
+ *          Transformer" (paper notes): sec. 3.2 "Linear Attention with RoPE"
+ *          (equation for O_i, linear-attention-with-RoPE pseudocode), sec. 3.4
+ *          "Block Linear Attention with Constant-Memory KV Cache" (causal
+ *          equation for O_i, cumulative state, Algorithm 1).
+ *   [SV2]  "SANA-Video 2.0" (hyper.ai summary), Method: hybrid attention and
+ *          block residuals, the AttnRes equation; shared router queries.
+ *   [SV2a] "SANA-Video 2.0" abstract: gated linear attention and gated softmax
+ *          anchors at a 3:1 ratio.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are row-major.  Token tensors are (B, N, C) with C = heads * D,
+ *     i.e. (B, N, heads, D) with D contiguous ([SV1] sec. 3.2 pseudocode
+ *     layout).  Token n of a latent grid (T, H, W) is n = (t*H + h)*W + w.
+ *   - Every pointer argument named "device" is CUDA device memory owned by the
+ *     caller; the library allocates no device memory and keeps no state between
+ *     calls except a thread-local error string and one device status word.
+ *   - Device pointers must be 16-byte aligned; outputs must not alias inputs
+ *     (SANA_ERR_INVALID_ARG otherwise).
+ *   - bf16 tensors use D = 128 (tcgen05 tensor-core path); fp32 tensors accept
+ *     D in {16, 32, 64, 128} (FFMA path).  Other D: SANA_ERR_UNSUPPORTED.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously.  Argument errors are returned before
+ *     anything is enqueued; launch errors return SANA_ERR_CUDA.  A kernel that
+ *     detects a fault (a bounded wait that ran out) records it in the device
+ *     status word, which sana_sync_status() reports as SANA_ERR_TIMEOUT.
+ *   - On any non-OK status, sana_last_error_string() describes the cause.
+ */
+#ifndef SANA_H_
+#define SANA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SANA_API __attribute__((visibility("default")))
+#else
+#define SANA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sana_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  SANA_OK = 0,
+  SANA_ERR_INVALID_ARG = 1,
+  SANA_ERR_UNSUPPORTED = 2,
+  SANA_ERR_WORKSPACE = 3,
+  SANA_ERR_CUDA = 4,
+  SANA_ERR_TIMEOUT = 5
+} sana_status;
+
+typedef enum { SANA_F32 = 0, SANA_BF16 = 1 } sana_dtype;
+
+/* Latent token grid of one call.  N = T*H*W tokens per batch entry.
+ * t_offset is the absolute index of the first frame (block-causal chunks use
+ * absolute frame positions for RoPE); 0 for whole clips. */
+typedef struct {
+  int B, T, H, W;
+  int heads, head_dim;
+  int t_offset;
+} sana_shape;
+
+/* 3D RoPE tables ([SV1] sec. 3.2, RoPE applied after the ReLU; layout reading:
+ * rotary pair j rotates elements (2j, 2j+1) of a head; pairs [0, n_t) follow
+ * the absolute frame index, the next n_h the row, the last n_w the column;
+ * n_t + n_h + n_w == head_dim / 2).  Device fp32 arrays, row-major:
+ * cos_t/sin_t [T_total][n_t], cos_h/sin_h [H][n_h], cos_w/sin_w [W][n_w]. */
+typedef struct {
+  const float *cos_t, *sin_t, *cos_h, *sin_h, *cos_w, *sin_w;
+  int n_t, n_h, n_w;
+  int T_total, H, W;
+} sana_rope;
+
+/* Number of floats sana_rope_tables_host() writes:
+ * 2*(T_total*n_t + H*n_h + W*n_w). */
+SANA_API size_t sana_rope_tables_count(int T_total, int H, int W, int n_t, int n_h, int n_w);
+
+/* Fill a HOST buffer with the six tables, in the order cos_t, sin_t, cos_h,
+ * sin_h, cos_w, sin_w; angle(pos, local pair k of an axis with n pairs) =
+ * pos * theta^(-k/n), evaluated in double and rounded to float.
+ * Errors: SANA_ERR_INVALID_ARG on a NULL buffer or negative sizes. */
+SANA_API sana_status sana_rope_tables_host(int T_total, int H, int W, int n_t, int n_h, int n_w,
+                                  double theta, float* out_tables_host);
+
+/* Point a sana_rope at a DEVICE copy of the buffer sana_rope_tables_host()
+ * filled (pointer arithmetic only; nothing is read). */
+SANA_API sana_status sana_rope_bind(const float* tables_device, int T_total, int H, int W,
+                           int n_t, int n_h, int n_w, sana_rope* out);
+
+/* ---------------------------------------------------------------------------
+ * Gated bidirectional ReLU linear attention with RoPE after the ReLU
+ * ([SV1] sec. 3.2):
+ *   S = sum_j RoPE(phi K_j)^T V_j,  z = sum_j phi K_j,  phi = ReLU,
+ *   O_i = RoPE(phi Q_i) S / (phi Q_i . z + eps),  Y_i = sigmoid(G_i) * O_i.
+ * q, k, v, gate_logits, out: device (B, N, C) in `dtype`; gate_logits may be
+ * NULL (no gate).  eps > 0.  ws: device workspace of at least
+ * sana_linattn_workspace_size() bytes (256-byte aligned), caller-owned,
+ * contents undefined on return.  The state reduction over N is split across
+ * CTAs and combined in a fixed order, so results are bit-reproducible.
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_linattn_workspace_size(const sana_shape* shape, sana_dtype dtype);
+SANA_API sana_status sana_linattn_fwd(const sana_shape* shape, sana_dtype dtype, const void* q,
+                             const void* k, const void* v, const void* gate_logits,
+                             const sana_rope* rope, float eps, void* out, void* ws,
+                             size_t ws_bytes, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The two halves of sana_linattn_fwd, callable on their own ([SV1] sec. 3.2
+ * pseudocode: the key-value contraction, then the query-side product and
+ * normalisation).
+ * sana_linattn_state: S_out = sum_j RoPE(phi K_j)^T V_j  (device fp32
+ *   [B][heads][D][D], S[d][e]) and z_out = sum_j phi K_j (device fp32
+ *   [B][heads][D]) over all N tokens.  Workspace:
+ *   sana_linattn_state_workspace_size() bytes (split partial sums).
+ * sana_linattn_apply: Y_i = sigmoid(G_i) * RoPE(phi Q_i) S / (phi Q_i . z + eps)
+ *   for a given state (S, z as above); needs no workspace.  For bf16 it is a
+ *   single kernel launch.
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_linattn_state_workspace_size(const sana_shape* shape, sana_dtype dtype);
+SANA_API sana_status sana_linattn_state(const sana_shape* shape, sana_dtype dtype, const void* k,
+                                        const void* v, const sana_rope* rope, float* S_out,
+                                        float* z_out, void* ws, size_t ws_bytes,
+                                        sana_stream_t stream);
+SANA_API sana_status sana_linattn_apply(const sana_shape* shape, sana_dtype dtype, const void* q,
+                                        const void* gate_logits, const sana_rope* rope,
+                                        const float* S, const float* z, float eps, void* out,
+                                        sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * One block of block-causal linear attention with the constant-memory state
+ * ([SV1] sec. 3.4 causal O_i and Algorithm 1).  shape describes the chunk
+ * (its T frames starting at absolute frame shape->t_offset).  The chunk's own
+ * (S_c, z_c) are added to the running state; its output uses
+ * (S_prev + S_c, z_prev + z_c): the chunk sees all earlier chunks and all of
+ * itself.  state_S: device fp32 [B][heads][D][D] (S[d][e] = sum RoPE(phi k)_d v_e),
+ * state_z: device fp32 [B][heads][D]; all-zero means "no past".  commit != 0
+ * writes the updated state back in place (Algorithm 1's cache update after the
+ * last denoising step); commit == 0 leaves it untouched.  Workspace as for
+ * sana_linattn_fwd (sana_linattn_workspace_size of the chunk shape).
+ * ------------------------------------------------------------------------- */
+SANA_API sana_status sana_linattn_block_causal_step(const sana_shape* chunk, sana_dtype dtype,
+                                           const void* q, const void* k, const void* v,
+                                           const void* gate_logits, const sana_rope* rope,
+                                           float eps, float* state_S, float* state_z,
+                                           int commit, void* out, void* ws, size_t ws_bytes,
+                                           sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Gated softmax anchor ([SV2a]; reading: the same 3D RoPE on raw Q, K):
+ *   Y = sigmoid(G) * softmax(RoPE(Q) RoPE(K)^T * scale) V, bidirectional over
+ *   all N keys of the same batch entry and head.
+ * rope may be NULL (no rotation).  scale <= 0 selects 1/sqrt(D).  Workspace:
+ * sana_softmax_anchor_workspace_size() bytes (rotated Q and K copies).
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_softmax_anchor_workspace_size(const sana_shape* shape, sana_dtype dtype);
+SANA_API sana_status sana_softmax_anchor_fwd(const sana_shape* shape, sana_dtype dtype, const void* q,
+                                    const void* k, const void* v, const void* gate_logits,
+                                    const sana_rope* rope, float scale, void* out, void* ws,
+                                    size_t ws_bytes, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Block Attention Residuals router ([SV2] AttnRes equation, timestep term 0):
+ *   l_i = w . v_i / sqrt(mean_c v_i^2 + rms_eps),  alpha = softmax_i(l),
+ *   h = sum_i alpha_i v_i,   per token, over num_sources sources.
+ * sources: HOST array of num_sources device pointers, each (B, N, C) in dtype,
+ * ordered [embedding, block summaries..., partial sum].  1 <= num_sources <= 16.
+ * w: device fp32 (C).  h_out: device (B, N, C) in dtype.  alpha_out: device
+ * fp32 (B, N, num_sources) or NULL.  C must be a multiple of 8.
+ * ------------------------------------------------------------------------- */
+SANA_API sana_status sana_attnres_route(int B, long long N, int C, sana_dtype dtype,
+                               const void* const* sources, int num_sources, const float* w,
+                               float rms_eps, void* h_out, float* alpha_out,
+                               sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Building blocks of the stack, exported for stage-wise checking.
+ * sana_gemm_bf16: out[M][N] = epilogue(A[M][K] . W[N][K]^T) with bf16 A, W, out
+ * and fp32 accumulation on tcgen05; epilogue 0 = identity, 1 = SiLU,
+ * 2 = out += result (residual add into out).  lda/ldo are row strides in
+ * elements (>= K / >= N, multiples of 8).  K must be a multiple of 64.
+ * sana_rmsnorm: y = x / sqrt(mean(x^2) + eps) per row (no gain), (rows, C).
+ * ------------------------------------------------------------------------- */
+typedef enum { SANA_EPI_NONE = 0, SANA_EPI_SILU = 1, SANA_EPI_RESIDUAL = 2 } sana_epilogue;
+SANA_API sana_status sana_gemm_bf16(long long M, int N, int K, const void* A, long long lda,
+                           const void* W, void* out, long long ldo, int epilogue,
+                           sana_stream_t stream);
+SANA_API sana_status sana_rmsnorm(long long rows, int C, sana_dtype dtype, const void* x, float eps,
+                         void* y, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Hybrid stack forward ([SV2] method; [SV2a] 3:1 interleave).
+ * Layer l (0-based) is a softmax anchor iff l % ratio == ratio - 1, else a
+ * gated linear-attention layer.  Each layer has an attention sublayer
+ * (RMSNorm -> x.W_qkvg^T split into Q, K, V, G -> gated attention -> .W_o^T)
+ * and, when ffn_mult > 0, an FFN sublayer (RMSNorm -> W_down SiLU(W_up x)).
+ * use_attnres != 0: each sublayer reads h = route(sources) with the shared
+ * attention or FFN query; its output is added to the running partial sum;
+ * every block_span layers the partial sum is frozen as a block summary; the
+ * result is route(final sources, w_attn).  use_attnres == 0: plain pre-norm
+ * residual x += sublayer(RMSNorm(x)); the result is the final x.
+ * bf16 only, D = 128, C = heads * 128.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int layers;
+  int block_span;
+  int ratio;
+  int use_attnres;
+  int ffn_mult;
+  float eps;          /* linear-attention denominator eps */
+  float rms_eps;      /* RMSNorm eps (routing and pre-norm) */
+  float anchor_scale; /* <= 0: 1/sqrt(D) */
+} sana_stack_config;
+
+typedef struct {
+  const void* const* w_qkvg; /* HOST array [layers] of device (4C, C) bf16 */
+  const void* const* w_o;    /* [layers] of (C, C) */
+  const void* const* w_up;   /* [layers] of (ffn_mult*C, C), or NULL if ffn_mult == 0 */
+  const void* const* w_down; /* [layers] of (C, ffn_mult*C), or NULL */
+  const float* w_attn;       /* device fp32 (C): shared attention router query */
+  const float* w_ffn;        /* device fp32 (C): shared FFN router query */
+} sana_stack_weights;
+
+SANA_API size_t sana_hybrid_stack_workspace_size(const sana_shape* shape, const sana_stack_config* cfg);
+SANA_API sana_status sana_hybrid_stack_fwd(const sana_shape* shape, const sana_stack_config* cfg,
+                                  const sana_stack_weights* weights, const sana_rope* rope,
+                                  const void* x_embed, void* out, void* ws, size_t ws_bytes,
+                                  sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Status helpers.
+ * sana_sync_status: synchronizes `stream`, then reports (and clears) the
+ * device status word: SANA_ERR_TIMEOUT if a kernel gave up a bounded wait,
+ * SANA_ERR_CUDA on an asynchronous CUDA error, else SANA_OK.
+ * sana_last_error_string: thread-local message of the last non-OK status.
+ * ------------------------------------------------------------------------- */
+SANA_API sana_status sana_sync_status(sana_stream_t stream);
+SANA_API const char* sana_last_error_string(void);
+SANA_API const char* sana_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SANA_H_ */

@@ -137,7 +137,7 @@ def linattn_state(k, v, angles, heads):
     vh = _heads(np.asarray(v, np.float64), heads)
     k_phi = phi(kh)
     k_rope = apply_rope(k_phi, angles)
-    S = np.einsum('bhnd,bhne->bhde', k_rope, vh)
+    S = np.swapaxes(k_rope, -1, -2) @ vh          # sum_j RoPE(phi K_j)^T V_j
     z = k_phi.sum(axis=2)
     return S, z
 
@@ -149,8 +149,8 @@ def linattn_apply(q, S, z, angles, heads, gate=None, eps=EPS):
     qh = _heads(np.asarray(q, np.float64), heads)
     q_phi = phi(qh)
     q_rope = apply_rope(q_phi, angles)
-    num = np.einsum('bhnd,bhde->bhne', q_rope, S)
-    den = np.einsum('bhnd,bhd->bhn', q_phi, z)
+    num = q_rope @ S                               # RoPE(phi Q_i) S
+    den = (q_phi @ z[..., :, None])[..., 0]        # phi Q_i . z
     out = _merge(num / (den[..., None] + eps))
     if gate is not None:
         out = sigmoid(np.asarray(gate, np.float64)) * out
@@ -266,11 +266,11 @@ def softmax_anchor(q, k, v, grid, rope_split, heads, gate=None, scale=None,
         kh = apply_rope(kh, ang)
     if rows is not None:
         qh = qh[:, :, rows]
-    logits = np.einsum('bhid,bhjd->bhij', qh, kh) * scale
+    logits = (qh @ np.swapaxes(kh, -1, -2)) * scale
     m = logits.max(axis=-1, keepdims=True)
     p = np.exp(logits - m)
     p = p / p.sum(axis=-1, keepdims=True)
-    out = _merge(np.einsum('bhij,bhjd->bhid', p, vh))
+    out = _merge(p @ vh)
     if gate is not None:
         g = np.asarray(gate, np.float64)
         if rows is not None:

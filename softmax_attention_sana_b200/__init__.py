@@ -1,0 +1,18 @@
+"""B200-native (sm_100a) hot path of SANA-Video 2.0's hybrid linear-softmax attention.
+
+The compute lives in libsana.so (C ABI declared in include/sana.h, kernels in
+csrc/); this package is a thin ctypes binding over it.
+"""
+
+from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_route, check,
+                   gemm_bf16, host_rope_tables, hybrid_stack_fwd, last_error, lib,
+                   linattn_apply, linattn_block_causal_step, linattn_fwd, linattn_state,
+                   linattn_workspace_size, rmsnorm,
+                   softmax_anchor_fwd, stack_config, sync_status)
+
+__all__ = [
+    "EPI_NONE", "EPI_RESIDUAL", "EPI_SILU", "Rope", "SanaError", "attnres_route", "check",
+    "gemm_bf16", "host_rope_tables", "hybrid_stack_fwd", "last_error", "lib",
+    "linattn_apply", "linattn_block_causal_step", "linattn_fwd", "linattn_state", "linattn_workspace_size", "rmsnorm",
+    "softmax_anchor_fwd", "stack_config", "sync_status",
+]

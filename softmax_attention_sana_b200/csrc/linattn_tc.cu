@@ -1,0 +1,563 @@
+// Gated ReLU linear attention with RoPE after the ReLU, bf16 on tcgen05.
+//
+//   "SANA-Video" paper notes, sec. 3.2 (equation for O_i, pseudocode):
+//     S = sum_j RoPE(phi K_j)^T V_j,  z = sum_j phi K_j,
+//     O_i = RoPE(phi Q_i) S / (phi Q_i . z + eps)
+//   sec. 3.4 (causal form, cumulative state S, z), Algorithm 1 (state update).
+//   "SANA-Video 2.0" abstract: gated linear attention; gate = sigmoid(G).
+//
+// Three kernels per call:
+//   state   per (batch, head, split): TMA K, V tiles (128 tokens x 128) ->
+//           ReLU + RoPE of K in shared memory (z accumulated on the way) ->
+//           tcgen05 D[d][e] += K'^T V with fp32 accumulation in TMEM ->
+//           partial S and z to the workspace.
+//   combine per (batch, head): fixed-order sum of the split partials (plus the
+//           carried state in block-causal mode) into S and z in fp32.
+//   output  per (batch, head, split): S (fp32) -> bf16 S^T operand in shared
+//           memory once per CTA; TMA Q, G tiles -> ReLU + RoPE of Q and the
+//           RoPE-free denominator phi(Q).z in registers -> tcgen05 D = Q' S ->
+//           epilogue divides, gates with sigmoid(G), stores bf16 through
+//           shared memory with TMA.
+#include <cuda.h>
+
+#include "rope_dev.cuh"
+#include "sana_common.cuh"
+#include "sana_internal.h"
+
+namespace sana {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kRows = 128;                // tokens per tile
+constexpr int kHalf = kRows * 64 * 2;     // one 64-column half of a tile: 16 KB
+constexpr int kTileB = 2 * kHalf;         // 32 KB
+constexpr int kWorkers = 256;             // 8 warps: (row quarter, column half)
+constexpr int kThreadsA = kWorkers + 64;  // + producer warp + MMA warp
+constexpr int kStagesA = 3;
+constexpr int kStagesQ = 3;
+constexpr int kStagesG = 2;
+constexpr int kThreadsB = kWorkers + 96;  // + Q producer, MMA, G producer
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// ReLU + RoPE of one 16-byte chunk (4 rotary pairs) of a swizzled tile row,
+// rewritten in place.  phi values are returned for z / the denominator.
+__device__ __forceinline__ void relu_rope_chunk(uint8_t* p, const RowRope& rr, int pair0,
+                                                float (&phi_out)[8]) {
+  uint4 raw = *reinterpret_cast<uint4*>(p);
+  uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 x = bf2_to_f2(w[i]);
+    x.x = fmaxf(x.x, 0.f);
+    x.y = fmaxf(x.y, 0.f);
+    phi_out[2 * i] = x.x;
+    phi_out[2 * i + 1] = x.y;
+    const float2 r = rotate(x.x, x.y, rr.cs(pair0 + i));
+    w[i] = f2_to_bf2(r.x, r.y);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ------------------------------------------------------------------------
+// state kernel
+// ------------------------------------------------------------------------
+struct StateSmemCtl {
+  uint64_t full[kStagesA];
+  uint64_t kready[kStagesA];
+  uint64_t empty[kStagesA];
+  uint64_t done;
+  uint32_t tmem;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+    linattn_state_kernel(const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, RopeDev rope, GridDev g,
+                         int tiles_total, int splits, float* __restrict__ ws_S,
+                         float* __restrict__ ws_z, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ StateSmemCtl ctl;
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* stages = smem;
+  float2* rope_base = reinterpret_cast<float2*>(smem + kStagesA * 2 * kTileB);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tile0 = (int)((long long)split * tiles_total / splits);
+  const int ntiles = (int)((long long)(split + 1) * tiles_total / splits) - tile0;
+  const WaitCtx wc{&ctl.abort_flag, status};
+  volatile int* abort_flag = &ctl.abort_flag;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStagesA; ++s) {
+      mbar_init(&ctl.full[s], 1);
+      mbar_init(&ctl.kready[s], kWorkers);
+      mbar_init(&ctl.empty[s], 1);
+    }
+    mbar_init(&ctl.done, 1);
+    ctl.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&ctl.tmem, 128);
+    tmem_relinquish();
+  }
+  const RopeSmem rs = rope_stage(rope_base, rope, g, tid, kThreadsA);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem;
+
+  if (warp == 8) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int issued = 0;
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kStagesA;
+        if (it >= kStagesA && !mbar_wait(&ctl.empty[s], ((it / kStagesA) - 1) & 1, wc, 0x11))
+          break;
+        const int n0 = (tile0 + it) * kRows;
+        uint8_t* st = stages + s * 2 * kTileB;
+        mbar_arrive_expect_tx(&ctl.full[s], 2 * kTileB);
+        tma_load_3d(st, &tm_k, &ctl.full[s], h * kD, n0, b);
+        tma_load_3d(st + kHalf, &tm_k, &ctl.full[s], h * kD + 64, n0, b);
+        tma_load_3d(st + kTileB, &tm_v, &ctl.full[s], h * kD, n0, b);
+        tma_load_3d(st + kTileB + kHalf, &tm_v, &ctl.full[s], h * kD + 64, n0, b);
+        ++issued;
+      }
+      if (*abort_flag) {  // drain loads still in flight before the CTA exits
+        for (int it = issued > kStagesA ? issued - kStagesA : 0; it < issued; ++it) {
+          mbar_drain(&ctl.full[it % kStagesA], (it / kStagesA) & 1);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer: D[d][e] += K'[tok][d]^T V[tok][e]
+    if (lane == 0) {
+      // A = K' (M = d, MN-major), B = V (N = e, MN-major), both 128B-swizzled
+      // [2 halves of 64][128 tokens]; LBO = distance of the 64-column halves,
+      // SBO = distance of 8-token groups.
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 1, 1);
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kStagesA;
+        if (!mbar_wait(&ctl.kready[s], (it / kStagesA) & 1, wc, 0x12)) break;
+        tc_fence_after();
+        const uint32_t kb = smem_u32(stages + s * 2 * kTileB);
+        const uint32_t vb = kb + kTileB;
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(kb + kk * 2048, kHalf, 1024);
+          const uint64_t bd = smem_desc_sw128(vb + kk * 2048, kHalf, 1024);
+          umma_ss(tmem, ad, bd, idesc, (it | kk) != 0);
+        }
+        umma_commit(&ctl.empty[s]);
+      }
+      umma_commit(&ctl.done);
+    }
+  } else {
+    // ---------------- workers: thread = (token row r, column half c)
+    const int q4 = warp & 3, c = warp >> 2, r = q4 * 32 + lane;
+    float zacc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) zacc[i] = 0.f;
+    for (int it = 0; it < ntiles; ++it) {
+      const int s = it % kStagesA;
+      if (!mbar_wait(&ctl.full[s], (it / kStagesA) & 1, wc, 0x13)) break;
+      const int n = (tile0 + it) * kRows + r;
+      if (n < g.N) {  // rows past N were zero-filled by TMA: phi = RoPE = 0
+        const RowRope rr = row_rope(rs, g, n);
+        uint8_t* half = stages + s * 2 * kTileB + c * kHalf;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          float ph[8];
+          relu_rope_chunk(half + sw128_off(r, ch), rr, c * 32 + ch * 4, ph);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) zacc[ch * 8 + i] += ph[i];
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&ctl.kready[s]);
+    }
+    const bool ok = mbar_wait(&ctl.done, 0, wc, 0x14);
+    tc_fence_after();
+    const size_t part = ((size_t)(b * g.heads + h) * splits + split);
+    if (ok) {
+      float* Sout = ws_S + part * kD * kD;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c * 64 + j * 32, v);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(Sout + (size_t)r * kD + c * 64 + j * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      }
+    }
+    // z: reduce the per-row partial sums over the 128 rows of each half in a
+    // fixed order (stride 65 keeps both passes free of bank conflicts).
+    float* red = reinterpret_cast<float*>(stages);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) red[(c * 128 + r) * 65 + i] = zacc[i];
+    named_bar_sync(1, kWorkers);
+    if (tid < 128) {
+      const int cc = tid >> 6, i = tid & 63;
+      float acc = 0.f;
+      for (int rr = 0; rr < 128; ++rr) acc += red[(cc * 128 + rr) * 65 + i];
+      ws_z[part * kD + cc * 64 + i] = acc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    if (*abort_flag) mbar_drain(&ctl.done, 0);  // MMAs in flight finish before TMEM is freed
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------------------
+// combine kernel (shared with the fp32 path): fixed-order sum over splits
+// ------------------------------------------------------------------------
+__global__ void linattn_combine_kernel(const float* __restrict__ ws_S,
+                                       const float* __restrict__ ws_z, int splits, int D,
+                                       const float* S_prev, const float* z_prev, float* S_state,
+                                       float* z_state, float* __restrict__ S_f32,
+                                       float* __restrict__ z_out) {
+  const int bh = blockIdx.x;
+  const size_t DD = (size_t)D * D;
+  for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x) {
+    float acc = S_prev ? S_prev[bh * DD + idx] : 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += ws_S[((size_t)bh * splits + sp) * DD + idx];
+    if (S_state) S_state[bh * DD + idx] = acc;
+    if (S_f32) S_f32[bh * DD + idx] = acc;
+  }
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = z_prev ? z_prev[(size_t)bh * D + d] : 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += ws_z[((size_t)bh * splits + sp) * D + d];
+    if (z_state) z_state[(size_t)bh * D + d] = acc;
+    if (z_out) z_out[(size_t)bh * D + d] = acc;
+  }
+}
+
+// ------------------------------------------------------------------------
+// output kernel
+// ------------------------------------------------------------------------
+struct OutSmemCtl {
+  uint64_t fullQ[kStagesQ], emptyQ[kStagesQ], qready[kStagesQ];
+  uint64_t fullG[kStagesG], emptyG[kStagesG];
+  uint64_t mma_done[2], tmem_free[2];
+  uint64_t wsync, hsync[2];  // reusable worker barriers (bounded waits)
+  uint32_t tmem;
+  int abort_flag;
+  float den[kStagesQ][2][kRows];
+  float z[kD];
+};
+
+template <bool kGate>
+__global__ void __launch_bounds__(kThreadsB, 1)
+    linattn_out_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_g,
+                       const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ S_all,
+                       const float* __restrict__ z_all, RopeDev rope, GridDev g, int tiles_total,
+                       int splits, float eps, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ OutSmemCtl ctl;
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* s_op = smem;                             // S^T operand, 32 KB
+  uint8_t* q_st = s_op + kTileB;                    // Q stages
+  uint8_t* g_st = q_st + kStagesQ * kTileB;         // G / Y stages
+  float2* rope_base = reinterpret_cast<float2*>(g_st + kStagesG * kTileB);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tile0 = (int)((long long)split * tiles_total / splits);
+  const int ntiles = (int)((long long)(split + 1) * tiles_total / splits) - tile0;
+  const int bh = b * g.heads + h;
+  const WaitCtx wc{&ctl.abort_flag, status};
+
+  if (tid == 0) {
+    for (int s = 0; s < kStagesQ; ++s) {
+      mbar_init(&ctl.fullQ[s], 1);
+      mbar_init(&ctl.emptyQ[s], 1);
+      mbar_init(&ctl.qready[s], kWorkers);
+    }
+    for (int s = 0; s < kStagesG; ++s) {
+      mbar_init(&ctl.fullG[s], 1);
+      mbar_init(&ctl.emptyG[s], 2);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl.mma_done[i], 1);
+      mbar_init(&ctl.tmem_free[i], kWorkers);
+      mbar_init(&ctl.hsync[i], 128);
+    }
+    mbar_init(&ctl.wsync, kWorkers);
+    ctl.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&ctl.tmem, 256);
+    tmem_relinquish();
+  }
+  if (tid < kD) ctl.z[tid] = z_all[(size_t)bh * kD + tid];
+  if (tid < kWorkers) {
+    // S^T operand: element (e, d) = S[d][e] in bf16, K-major [2 halves of
+    // 64 d][128 e rows] with the 128-byte swizzle.  Thread = (row e, half).
+    const int e = tid & 127, hf = tid >> 7;
+    const float* Sh = S_all + (size_t)bh * kD * kD + (size_t)(hf * 64) * kD + e;
+    uint8_t* dst = s_op + hf * kHalf;
+#pragma unroll 2
+    for (int ch = 0; ch < 8; ++ch) {
+      uint32_t wv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        wv[i] = f2_to_bf2(Sh[(ch * 8 + 2 * i) * kD], Sh[(ch * 8 + 2 * i + 1) * kD]);
+      *reinterpret_cast<uint4*>(dst + sw128_off(e, ch)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+    fence_proxy_async_smem();
+  }
+  const RopeSmem rs = rope_stage(rope_base, rope, g, tid, kThreadsB);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem;
+
+  if (warp == 8) {
+    // ---------------- Q producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kStagesQ;
+        if (it >= kStagesQ && !mbar_wait(&ctl.emptyQ[s], ((it / kStagesQ) - 1) & 1, wc, 0x21))
+          break;
+        const int n0 = (tile0 + it) * kRows;
+        mbar_arrive_expect_tx(&ctl.fullQ[s], kTileB);
+        tma_load_3d(q_st + s * kTileB, &tm_q, &ctl.fullQ[s], h * kD, n0, b);
+        tma_load_3d(q_st + s * kTileB + kHalf, &tm_q, &ctl.fullQ[s], h * kD + 64, n0, b);
+      }
+    }
+  } else if (warp == 10) {
+    // ---------------- G producer (ungated: only hands out the staging buffers)
+    if (lane == 0) {
+      if (kGate) prefetch_tmap(&tm_g);
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kStagesG;
+        if (it >= kStagesG && !mbar_wait(&ctl.emptyG[s], ((it / kStagesG) - 1) & 1, wc, 0x22))
+          break;
+        if (kGate) {
+          const int n0 = (tile0 + it) * kRows;
+          mbar_arrive_expect_tx(&ctl.fullG[s], kTileB);
+          tma_load_3d(g_st + s * kTileB, &tm_g, &ctl.fullG[s], h * kD, n0, b);
+          tma_load_3d(g_st + s * kTileB + kHalf, &tm_g, &ctl.fullG[s], h * kD + 64, n0, b);
+        } else {
+          mbar_arrive(&ctl.fullG[s]);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer: D[tok][e] = Q'[tok][d] S[d][e]
+    if (lane == 0) {
+      // A = Q' (K-major, [2 halves][128 tok][64 d]), B = S^T (K-major,
+      // [2 halves][128 e][64 d]); a K step of 16 advances 32 bytes in a half.
+      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t sb = smem_u32(s_op);
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kStagesQ, tb = it & 1;
+        if (!mbar_wait(&ctl.qready[s], (it / kStagesQ) & 1, wc, 0x24)) break;
+        if (it >= 2 && !mbar_wait(&ctl.tmem_free[tb], ((it >> 1) - 1) & 1, wc, 0x25)) break;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(q_st + s * kTileB);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          umma_ss(tmem + tb * 128, smem_desc_sw128(qb + off, 16, 1024),
+                  smem_desc_sw128(sb + off, 16, 1024), idesc, kk != 0);
+        }
+        umma_commit(&ctl.emptyQ[s]);
+        umma_commit(&ctl.mma_done[tb]);
+      }
+    }
+  } else {
+    // ---------------- workers: thread = (token row r, column half c)
+    const int q4 = warp & 3, c = warp >> 2, r = q4 * 32 + lane;
+    bool ok = true;
+    auto prologue = [&](int it) {
+      const int s = it % kStagesQ;
+      if (!mbar_wait(&ctl.fullQ[s], (it / kStagesQ) & 1, wc, 0x26)) {
+        ok = false;
+        return;
+      }
+      const int n = (tile0 + it) * kRows + r;
+      float den = 0.f;
+      if (n < g.N) {
+        const RowRope rr = row_rope(rs, g, n);
+        uint8_t* half = q_st + s * kTileB + c * kHalf;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          float ph[8];
+          relu_rope_chunk(half + sw128_off(r, ch), rr, c * 32 + ch * 4, ph);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) den = fmaf(ph[i], ctl.z[c * 64 + ch * 8 + i], den);
+        }
+      }
+      ctl.den[s][c][r] = den;
+      fence_proxy_async_smem();
+      mbar_arrive(&ctl.qready[s]);
+    };
+    uint32_t n_wsync = 0, n_hsync = 0;
+    auto epilogue = [&](int it) {
+      const int s = it % kStagesQ, tb = it & 1, sg = it % kStagesG;
+      bool okw = mbar_wait(&ctl.mma_done[tb], (it >> 1) & 1, wc, 0x27);
+      // both column halves have written their partial denominators
+      mbar_arrive(&ctl.wsync);
+      okw = mbar_wait(&ctl.wsync, (n_wsync++) & 1, wc, 0x29) && okw;
+      const float inv = 1.f / (ctl.den[s][0][r] + ctl.den[s][1][r] + eps);
+      uint32_t acc[2][32];
+      if (okw) {
+        tc_fence_after();
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 128 + c * 64, acc[0]);
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 128 + c * 64 + 32, acc[1]);
+        tmem_ld_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl.tmem_free[tb]);
+      okw = mbar_wait(&ctl.fullG[sg], (it / kStagesG) & 1, wc, 0x28) && okw;
+      uint8_t* half = g_st + sg * kTileB + c * kHalf;
+      if (okw) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4* p = reinterpret_cast<uint4*>(half + sw128_off(r, ch));
+          uint32_t gw[4] = {0, 0, 0, 0};
+          if (kGate) {
+            const uint4 graw = *p;
+            gw[0] = graw.x; gw[1] = graw.y; gw[2] = graw.z; gw[3] = graw.w;
+          }
+          uint32_t out[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int col = (ch & 3) * 8 + 2 * i;
+            float y0 = __uint_as_float(acc[ch >> 2][col]) * inv;
+            float y1 = __uint_as_float(acc[ch >> 2][col + 1]) * inv;
+            if (kGate) {
+              const float2 gg = bf2_to_f2(gw[i]);
+              y0 *= sigmoid_fast(gg.x);
+              y1 *= sigmoid_fast(gg.y);
+            }
+            out[i] = f2_to_bf2(y0, y1);
+          }
+          *p = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      // the 128 rows of this column half are staged
+      mbar_arrive(&ctl.hsync[c]);
+      okw = mbar_wait(&ctl.hsync[c], (n_hsync++) & 1, wc, 0x2a) && okw;
+      if (okw && q4 == 0 && lane == 0) {
+        tma_store_3d(&tm_y, half, h * kD + c * 64, (tile0 + it) * kRows, b);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(&ctl.emptyG[sg]);
+      }
+      ok = okw;
+    };
+    if (ntiles > 0) prologue(0);
+    for (int it = 0; ok && it < ntiles; ++it) {
+      if (it + 1 < ntiles) prologue(it + 1);
+      if (!ok) break;
+      epilogue(it);
+    }
+    if (q4 == 0 && lane == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+constexpr size_t kStateSmem = 1024 + kStagesA * 2 * kTileB;
+constexpr size_t kOutSmem = 1024 + kTileB + kStagesQ * kTileB + kStagesG * kTileB;
+
+}  // namespace
+
+// ------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------
+namespace {
+void set_smem_attrs() {
+  static bool done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || done[dev]) return;
+  cudaFuncSetAttribute(linattn_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)(kStateSmem + kRopeSmemMax));
+  cudaFuncSetAttribute(linattn_out_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)(kOutSmem + kRopeSmemMax));
+  cudaFuncSetAttribute(linattn_out_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)(kOutSmem + kRopeSmemMax));
+  done[dev] = true;
+}
+}  // namespace
+
+// State phase: split reduction + fixed-order combine into S_f32 / z_out
+// (and the carried state when committing).
+sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, const void* k,
+                               const void* v, const RopeDev& rope, const GridDev& g,
+                               const float* S_prev, const float* z_prev, float* S_state,
+                               float* z_state, float* ws_S, float* ws_z, float* S_f32,
+                               float* z_out, cudaStream_t st) {
+  const uint64_t C = (uint64_t)s.heads * kD, N = (uint64_t)g.N;
+  CUtensorMap tk, tv;
+  if (!make_tmap_bf16_3d(&tk, k, C, N, s.B, C, N * C, kRows) ||
+      !make_tmap_bf16_3d(&tv, v, C, N, s.B, C, N * C, kRows))
+    return fail(SANA_ERR_CUDA, "linattn: cuTensorMapEncodeTiled failed");
+  set_smem_attrs();
+  const size_t smem_a = kStateSmem + rope_smem_bytes(g, rope);
+  linattn_state_kernel<<<dim3(plan.splits_a, s.heads, s.B), kThreadsA, smem_a, st>>>(
+      tk, tv, rope, g, plan.tiles, plan.splits_a, ws_S, ws_z, status_word());
+  if (sana_status e = check_launch("linattn_state_kernel")) return e;
+  linattn_combine_kernel<<<s.B * s.heads, 256, 0, st>>>(ws_S, ws_z, plan.splits_a, kD, S_prev,
+                                                        z_prev, S_state, z_state, S_f32, z_out);
+  return check_launch("linattn_combine_kernel");
+}
+
+// Output phase: one kernel launch.
+sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, const void* q,
+                               const void* gt, const RopeDev& rope, const GridDev& g,
+                               const float* S_f32, const float* z, float eps, void* out,
+                               cudaStream_t st) {
+  const uint64_t C = (uint64_t)s.heads * kD, N = (uint64_t)g.N;
+  CUtensorMap tq, tg, ty;
+  bool okm = make_tmap_bf16_3d(&tq, q, C, N, s.B, C, N * C, kRows) &&
+             make_tmap_bf16_3d(&ty, out, C, N, s.B, C, N * C, kRows);
+  if (gt) okm = okm && make_tmap_bf16_3d(&tg, gt, C, N, s.B, C, N * C, kRows);
+  else tg = tq;
+  if (!okm) return fail(SANA_ERR_CUDA, "linattn: cuTensorMapEncodeTiled failed");
+  set_smem_attrs();
+  const size_t smem_b = kOutSmem + rope_smem_bytes(g, rope);
+  if (gt)
+    linattn_out_kernel<true><<<dim3(plan.splits_b, s.heads, s.B), kThreadsB, smem_b, st>>>(
+        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, status_word());
+  else
+    linattn_out_kernel<false><<<dim3(plan.splits_b, s.heads, s.B), kThreadsB, smem_b, st>>>(
+        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, status_word());
+  return check_launch("linattn_out_kernel");
+}
+
+// The fp32 path reuses the combine kernel.
+void launch_linattn_combine(int BH, const float* ws_S, const float* ws_z, int splits, int D,
+                            const float* S_prev, const float* z_prev, float* S_state,
+                            float* z_state, float* S_f32, float* z_out, cudaStream_t st) {
+  linattn_combine_kernel<<<BH, 256, 0, st>>>(ws_S, ws_z, splits, D, S_prev, z_prev, S_state,
+                                             z_state, S_f32, z_out);
+}
+
+}  // namespace sana

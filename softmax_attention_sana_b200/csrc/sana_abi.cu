@@ -1,0 +1,590 @@
+// libsana C ABI: argument validation, workspace sizing, dispatch to the
+// kernels, RoPE tables, error strings and the device status word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "sana_common.cuh"
+#include "sana_internal.h"
+
+namespace sana {
+
+__device__ int g_status_word;
+
+namespace {
+thread_local std::string g_err = "ok";
+}
+
+sana_status fail(sana_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+sana_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SANA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return SANA_OK;
+}
+
+int* status_word() {
+  static int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+// ---------------------------------------------------------------- tensor maps
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                       uint64_t batches, uint64_t row_stride, uint64_t batch_stride,
+                       uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {cols, rows, batches};
+  const cuuint64_t strides[2] = {row_stride * 2, batch_stride * 2};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                       uint64_t row_stride, uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- validation helpers
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+size_t esize(sana_dtype dt) { return dt == SANA_BF16 ? 2 : 4; }
+
+sana_status check_shape(const sana_shape* s, sana_dtype dt, const char* who) {
+  if (!s) return fail(SANA_ERR_INVALID_ARG, "%s: shape is NULL", who);
+  if (dt != SANA_F32 && dt != SANA_BF16) return fail(SANA_ERR_INVALID_ARG, "%s: bad dtype %d", who, (int)dt);
+  if (s->B < 1 || s->T < 0 || s->H < 1 || s->W < 1 || s->heads < 1 || s->t_offset < 0)
+    return fail(SANA_ERR_INVALID_ARG, "%s: bad shape B=%d T=%d H=%d W=%d heads=%d t_offset=%d", who,
+                s->B, s->T, s->H, s->W, s->heads, s->t_offset);
+  const long long N = (long long)s->T * s->H * s->W;
+  if (N >= (1LL << 31) / 2) return fail(SANA_ERR_UNSUPPORTED, "%s: N=%lld too large", who, N);
+  const int D = s->head_dim;
+  if (dt == SANA_BF16 && D != 128)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: bf16 needs head_dim 128 (got %d)", who, D);
+  if (dt == SANA_F32 && D != 16 && D != 32 && D != 64 && D != 128)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: fp32 head_dim must be 16/32/64/128 (got %d)", who, D);
+  return SANA_OK;
+}
+
+sana_status check_rope(const sana_rope* r, const sana_shape* s, const char* who) {
+  if (!r) return fail(SANA_ERR_INVALID_ARG, "%s: rope is NULL", who);
+  if (r->n_t < 0 || r->n_h < 0 || r->n_w < 0 || r->n_t + r->n_h + r->n_w != s->head_dim / 2)
+    return fail(SANA_ERR_INVALID_ARG, "%s: rope split %d/%d/%d does not cover head_dim/2=%d", who,
+                r->n_t, r->n_h, r->n_w, s->head_dim / 2);
+  if (r->H != s->H || r->W != s->W || r->T_total < s->t_offset + s->T)
+    return fail(SANA_ERR_INVALID_ARG,
+                "%s: rope tables (T_total=%d, H=%d, W=%d) do not cover frames [%d, %d) of %dx%d", who,
+                r->T_total, r->H, r->W, s->t_offset, s->t_offset + s->T, s->H, s->W);
+  if ((r->n_t && (!r->cos_t || !r->sin_t)) || (r->n_h && (!r->cos_h || !r->sin_h)) ||
+      (r->n_w && (!r->cos_w || !r->sin_w)))
+    return fail(SANA_ERR_INVALID_ARG, "%s: rope table pointer is NULL", who);
+  return SANA_OK;
+}
+
+RopeDev to_dev(const sana_rope& r) {
+  return RopeDev{r.cos_t, r.sin_t, r.cos_h, r.sin_h, r.cos_w, r.sin_w, r.n_t, r.n_h, r.n_w};
+}
+
+GridDev to_grid(const sana_shape& s) {
+  return GridDev{s.T, s.H, s.W, s.t_offset, s.T * s.H * s.W, s.heads};
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- linear attention
+sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, const void* k,
+                               const void* v, const RopeDev& rope, const GridDev& g,
+                               const float* S_prev, const float* z_prev, float* S_state,
+                               float* z_state, float* ws_S, float* ws_z, float* S_f32,
+                               float* z_out, cudaStream_t st);
+sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, const void* q,
+                               const void* gt, const RopeDev& rope, const GridDev& g,
+                               const float* S_f32, const float* z, float eps, void* out,
+                               cudaStream_t st);
+int linattn_f32_splits(const sana_shape& s, int N);
+sana_status linattn_f32_state(const sana_shape& s, const float* k, const float* v,
+                              const RopeDev& rope, const GridDev& g, int splits,
+                              const float* S_prev, const float* z_prev, float* S_state,
+                              float* z_state, float* ws_S, float* ws_z, float* S_f32,
+                              float* z_comb, cudaStream_t st);
+sana_status linattn_f32_apply(const sana_shape& s, const float* q, const float* gt,
+                              const RopeDev& rope, const GridDev& g, const float* S_f32,
+                              const float* z, float eps, float* out, cudaStream_t st);
+
+LinAttnPlan linattn_plan(const sana_shape& s, sana_dtype dt) {
+  LinAttnPlan p{};
+  const int N = s.T * s.H * s.W;
+  const int bh = s.B * s.heads;
+  if (dt == SANA_BF16) {
+    p.tiles = (N + 127) / 128;
+    int sp = kNumSMs / bh;
+    if (sp < 1) sp = 1;
+    if (sp > p.tiles) sp = p.tiles;
+    if (sp < 1) sp = 1;
+    p.splits_a = p.splits_b = sp;
+  } else {
+    p.tiles = (N + 31) / 32;
+    p.splits_a = p.splits_b = linattn_f32_splits(s, N > 0 ? N : 1);
+  }
+  return p;
+}
+
+namespace {
+struct LinWs {
+  float* ws_S;   // split partials of S
+  float* ws_z;   // split partials of z
+  float* S_f32;  // combined S
+  float* z_comb; // combined z
+  size_t partial_bytes;  // what the state phase alone needs
+  size_t bytes;          // what the whole layer needs
+};
+LinWs carve_linattn(const sana_shape& s, sana_dtype dt, void* ws) {
+  const LinAttnPlan p = linattn_plan(s, dt);
+  const size_t bh = (size_t)s.B * s.heads, D = s.head_dim;
+  Carver cv(ws, ~size_t(0));
+  LinWs w{};
+  w.ws_S = cv.take<float>(bh * p.splits_a * D * D);
+  w.ws_z = cv.take<float>(bh * p.splits_a * D);
+  w.partial_bytes = align_up(cv.used, 256);
+  w.S_f32 = cv.take<float>(bh * D * D);
+  w.z_comb = cv.take<float>(bh * D);
+  w.bytes = align_up(cv.used, 256);
+  return w;
+}
+
+sana_status state_phase(const sana_shape& s, sana_dtype dt, const void* k, const void* v,
+                        const RopeDev& rope, const GridDev& g, const float* S_prev,
+                        const float* z_prev, float* S_state, float* z_state, const LinWs& w,
+                        float* S_out, float* z_out, cudaStream_t st) {
+  const LinAttnPlan p = linattn_plan(s, dt);
+  if (dt == SANA_BF16)
+    return linattn_bf16_state(s, p, k, v, rope, g, S_prev, z_prev, S_state, z_state, w.ws_S,
+                              w.ws_z, S_out, z_out, st);
+  return linattn_f32_state(s, static_cast<const float*>(k), static_cast<const float*>(v), rope, g,
+                           p.splits_a, S_prev, z_prev, S_state, z_state, w.ws_S, w.ws_z, S_out,
+                           z_out, st);
+}
+
+sana_status apply_phase(const sana_shape& s, sana_dtype dt, const void* q, const void* gt,
+                        const RopeDev& rope, const GridDev& g, const float* S, const float* z,
+                        float eps, void* out, cudaStream_t st) {
+  if (dt == SANA_BF16) {
+    if (rope_smem_bytes(g, rope) > kRopeSmemMax)
+      return fail(SANA_ERR_UNSUPPORTED,
+                  "linear attention: grid %dx%dx%d needs %zu B of RoPE tables (max %zu)", g.T, g.H,
+                  g.W, rope_smem_bytes(g, rope), kRopeSmemMax);
+    return linattn_bf16_apply(s, linattn_plan(s, dt), q, gt, rope, g, S, z, eps, out, st);
+  }
+  return linattn_f32_apply(s, static_cast<const float*>(q), static_cast<const float*>(gt), rope,
+                           g, S, z, eps, static_cast<float*>(out), st);
+}
+}  // namespace
+
+size_t linattn_ws_bytes(const sana_shape& s, sana_dtype dt) {
+  return carve_linattn(s, dt, nullptr).bytes;
+}
+size_t linattn_state_ws_bytes(const sana_shape& s, sana_dtype dt) {
+  return carve_linattn(s, dt, nullptr).partial_bytes;
+}
+
+sana_status linattn_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,
+                        const void* v, const void* gt, const RopeDev& rope, float eps,
+                        float* state_S, float* state_z, bool causal, bool commit, void* out,
+                        void* ws, size_t ws_bytes, cudaStream_t st) {
+  const GridDev g = to_grid(s);
+  if (g.N == 0) return SANA_OK;
+  const LinWs w = carve_linattn(s, dt, ws);
+  if (ws_bytes < w.bytes)
+    return fail(SANA_ERR_WORKSPACE, "linear attention: workspace %zu < %zu bytes", ws_bytes, w.bytes);
+  if (dt == SANA_BF16 && rope_smem_bytes(g, rope) > kRopeSmemMax)
+    return fail(SANA_ERR_UNSUPPORTED,
+                "linear attention: grid %dx%dx%d needs %zu B of RoPE tables (max %zu)", g.T, g.H,
+                g.W, rope_smem_bytes(g, rope), kRopeSmemMax);
+  const float* S_prev = causal ? state_S : nullptr;
+  const float* z_prev = causal ? state_z : nullptr;
+  float* S_commit = causal && commit ? state_S : nullptr;
+  float* z_commit = causal && commit ? state_z : nullptr;
+  if (sana_status e = state_phase(s, dt, k, v, rope, g, S_prev, z_prev, S_commit, z_commit, w,
+                                  w.S_f32, w.z_comb, st))
+    return e;
+  return apply_phase(s, dt, q, gt, rope, g, w.S_f32, w.z_comb, eps, out, st);
+}
+
+sana_status linattn_state_run(const sana_shape& s, sana_dtype dt, const void* k, const void* v,
+                              const RopeDev& rope, float* S_out, float* z_out, void* ws,
+                              size_t ws_bytes, cudaStream_t st) {
+  const GridDev g = to_grid(s);
+  const LinWs w = carve_linattn(s, dt, ws);
+  if (ws_bytes < w.partial_bytes)
+    return fail(SANA_ERR_WORKSPACE, "linear attention state: workspace %zu < %zu bytes", ws_bytes,
+                w.partial_bytes);
+  if (g.N == 0) {
+    cudaMemsetAsync(S_out, 0, (size_t)s.B * s.heads * s.head_dim * s.head_dim * 4, st);
+    cudaMemsetAsync(z_out, 0, (size_t)s.B * s.heads * s.head_dim * 4, st);
+    return check_launch("linear attention state (empty)");
+  }
+  if (dt == SANA_BF16 && rope_smem_bytes(g, rope) > kRopeSmemMax)
+    return fail(SANA_ERR_UNSUPPORTED, "linear attention: grid needs too many RoPE table bytes");
+  return state_phase(s, dt, k, v, rope, g, nullptr, nullptr, nullptr, nullptr, w, S_out, z_out, st);
+}
+
+sana_status linattn_apply_run(const sana_shape& s, sana_dtype dt, const void* q, const void* gt,
+                              const RopeDev& rope, const float* S, const float* z, float eps,
+                              void* out, cudaStream_t st) {
+  const GridDev g = to_grid(s);
+  if (g.N == 0) return SANA_OK;
+  return apply_phase(s, dt, q, gt, rope, g, S, z, eps, out, st);
+}
+
+// ---------------------------------------------------------------- anchor
+sana_status rope_rotate_run(const void* x, bool bf16, const RopeDev* rope, const GridDev& g, int B,
+                            int D, float mul, void* out, cudaStream_t st);
+sana_status anchor_f32_run(const sana_shape& s, const float* qr, const float* kr, const float* v,
+                           const float* gt, const GridDev& g, float scale, float* out,
+                           cudaStream_t st);
+sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr, const void* v,
+                            const void* gt, const GridDev& g, void* out, cudaStream_t st);
+
+size_t anchor_ws_bytes(const sana_shape& s, sana_dtype dt) {
+  const size_t n = (size_t)s.B * s.T * s.H * s.W * s.heads * s.head_dim;
+  Carver cv(nullptr, ~size_t(0));
+  cv.take<char>(n * esize(dt));
+  cv.take<char>(n * esize(dt));
+  return align_up(cv.used, 256);
+}
+
+sana_status anchor_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,
+                       const void* v, const void* gt, const RopeDev* rope, float scale, void* out,
+                       void* ws, size_t ws_bytes, cudaStream_t st) {
+  const GridDev g = to_grid(s);
+  if (g.N == 0) return SANA_OK;
+  const size_t need = anchor_ws_bytes(s, dt);
+  if (ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "softmax anchor: workspace %zu < %zu bytes", ws_bytes, need);
+  const size_t n = (size_t)s.B * g.N * s.heads * s.head_dim;
+  Carver cv(ws, ws_bytes);
+  void* qr = cv.take<char>(n * esize(dt));
+  void* kr = cv.take<char>(n * esize(dt));
+  const int D = s.head_dim;
+  if (scale <= 0.f) scale = 1.f / sqrtf((float)D);
+  if (dt == SANA_BF16) {
+    // Q is pre-scaled by scale * log2(e) so the kernel's softmax works in base 2.
+    const float qmul = scale * 1.4426950408889634f;
+    if (sana_status e = rope_rotate_run(q, true, rope, g, s.B, D, qmul, qr, st)) return e;
+    if (sana_status e = rope_rotate_run(k, true, rope, g, s.B, D, 1.f, kr, st)) return e;
+    return anchor_bf16_run(s, qr, kr, v, gt, g, out, st);
+  }
+  if (sana_status e = rope_rotate_run(q, false, rope, g, s.B, D, 1.f, qr, st)) return e;
+  if (sana_status e = rope_rotate_run(k, false, rope, g, s.B, D, 1.f, kr, st)) return e;
+  return anchor_f32_run(s, static_cast<const float*>(qr), static_cast<const float*>(kr),
+                        static_cast<const float*>(v), static_cast<const float*>(gt), g, scale,
+                        static_cast<float*>(out), st);
+}
+
+}  // namespace sana
+
+// ============================================================================
+// extern "C" entry points
+// ============================================================================
+using namespace sana;
+
+extern "C" {
+
+const char* sana_version(void) { return "libsana 0.1 (sm_100a)"; }
+
+const char* sana_last_error_string(void) { return g_err.c_str(); }
+
+size_t sana_rope_tables_count(int T_total, int H, int W, int n_t, int n_h, int n_w) {
+  if (T_total < 0 || H < 0 || W < 0 || n_t < 0 || n_h < 0 || n_w < 0) return 0;
+  return 2 * ((size_t)T_total * n_t + (size_t)H * n_h + (size_t)W * n_w);
+}
+
+sana_status sana_rope_tables_host(int T_total, int H, int W, int n_t, int n_h, int n_w,
+                                  double theta, float* out) {
+  if (!out) return fail(SANA_ERR_INVALID_ARG, "rope tables: output buffer is NULL");
+  if (T_total < 0 || H < 0 || W < 0 || n_t < 0 || n_h < 0 || n_w < 0 || !(theta > 0.0))
+    return fail(SANA_ERR_INVALID_ARG, "rope tables: bad sizes or theta");
+  float* p = out;
+  const int npos[3] = {T_total, H, W};
+  const int npair[3] = {n_t, n_h, n_w};
+  for (int ax = 0; ax < 3; ++ax) {
+    float* c = p;
+    float* s = p + (size_t)npos[ax] * npair[ax];
+    for (int pos = 0; pos < npos[ax]; ++pos)
+      for (int k = 0; k < npair[ax]; ++k) {
+        const double ang = (double)pos * std::pow(theta, -(double)k / npair[ax]);
+        c[(size_t)pos * npair[ax] + k] = (float)std::cos(ang);
+        s[(size_t)pos * npair[ax] + k] = (float)std::sin(ang);
+      }
+    p += 2 * (size_t)npos[ax] * npair[ax];
+  }
+  return SANA_OK;
+}
+
+sana_status sana_rope_bind(const float* t, int T_total, int H, int W, int n_t, int n_h, int n_w,
+                           sana_rope* out) {
+  if (!t || !out) return fail(SANA_ERR_INVALID_ARG, "rope bind: NULL argument");
+  if (T_total < 0 || H < 0 || W < 0 || n_t < 0 || n_h < 0 || n_w < 0)
+    return fail(SANA_ERR_INVALID_ARG, "rope bind: bad sizes");
+  out->cos_t = t;
+  out->sin_t = t + (size_t)T_total * n_t;
+  t += 2 * (size_t)T_total * n_t;
+  out->cos_h = t;
+  out->sin_h = t + (size_t)H * n_h;
+  t += 2 * (size_t)H * n_h;
+  out->cos_w = t;
+  out->sin_w = t + (size_t)W * n_w;
+  out->n_t = n_t;
+  out->n_h = n_h;
+  out->n_w = n_w;
+  out->T_total = T_total;
+  out->H = H;
+  out->W = W;
+  return SANA_OK;
+}
+
+size_t sana_linattn_workspace_size(const sana_shape* s, sana_dtype dt) {
+  if (check_shape(s, dt, "sana_linattn_workspace_size") != SANA_OK) return 0;
+  return linattn_ws_bytes(*s, dt);
+}
+
+static sana_status linattn_common(const char* who, const sana_shape* s, sana_dtype dt,
+                                  const void* q, const void* k, const void* v, const void* g,
+                                  const sana_rope* rope, float eps, float* S, float* z,
+                                  bool causal, int commit, void* out, void* ws, size_t ws_bytes,
+                                  sana_stream_t stream) {
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  if (!std::isfinite(eps) || eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", who);
+  const void* ptrs[5] = {q, k, v, g, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
+  if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, g, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an input", who);
+  if (causal) {
+    if (!S || !z) return fail(SANA_ERR_INVALID_ARG, "%s: state pointers are NULL", who);
+    const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
+    const size_t zb = (size_t)s->B * s->heads * s->head_dim * 4;
+    if (overlap(S, sb, out, n) || overlap(z, zb, out, n) || overlap(S, sb, z, zb))
+      return fail(SANA_ERR_INVALID_ARG, "%s: state aliases the output", who);
+    if (!aligned16(S) || !aligned16(z)) return fail(SANA_ERR_INVALID_ARG, "%s: state must be 16-byte aligned", who);
+  }
+  const size_t need = linattn_ws_bytes(*s, dt);
+  if (need && (!ws || ws_bytes < need))
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  return linattn_run(*s, dt, q, k, v, g, to_dev(*rope), eps, S, z, causal, commit != 0, out, ws,
+                     ws_bytes, stream);
+}
+
+sana_status sana_linattn_fwd(const sana_shape* s, sana_dtype dt, const void* q, const void* k,
+                             const void* v, const void* g, const sana_rope* rope, float eps,
+                             void* out, void* ws, size_t ws_bytes, sana_stream_t stream) {
+  return linattn_common("sana_linattn_fwd", s, dt, q, k, v, g, rope, eps, nullptr, nullptr, false,
+                        0, out, ws, ws_bytes, stream);
+}
+
+sana_status sana_linattn_block_causal_step(const sana_shape* s, sana_dtype dt, const void* q,
+                                           const void* k, const void* v, const void* g,
+                                           const sana_rope* rope, float eps, float* S, float* z,
+                                           int commit, void* out, void* ws, size_t ws_bytes,
+                                           sana_stream_t stream) {
+  return linattn_common("sana_linattn_block_causal_step", s, dt, q, k, v, g, rope, eps, S, z, true,
+                        commit, out, ws, ws_bytes, stream);
+}
+
+size_t sana_linattn_state_workspace_size(const sana_shape* s, sana_dtype dt) {
+  if (check_shape(s, dt, "sana_linattn_state_workspace_size") != SANA_OK) return 0;
+  return linattn_state_ws_bytes(*s, dt);
+}
+
+sana_status sana_linattn_state(const sana_shape* s, sana_dtype dt, const void* k, const void* v,
+                               const sana_rope* rope, float* S_out, float* z_out, void* ws,
+                               size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_linattn_state";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!k || !v || !S_out || !z_out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  const void* ptrs[4] = {k, v, S_out, z_out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
+  const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
+  const size_t zb = (size_t)s->B * s->heads * s->head_dim * 4;
+  if (overlap(S_out, sb, k, n) || overlap(S_out, sb, v, n) || overlap(z_out, zb, k, n) ||
+      overlap(z_out, zb, v, n) || overlap(S_out, sb, z_out, zb))
+    return fail(SANA_ERR_INVALID_ARG, "%s: outputs alias inputs", who);
+  const size_t need = linattn_state_ws_bytes(*s, dt);
+  if (need && (!ws || ws_bytes < need))
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  return linattn_state_run(*s, dt, k, v, to_dev(*rope), S_out, z_out, ws, ws_bytes, stream);
+}
+
+sana_status sana_linattn_apply(const sana_shape* s, sana_dtype dt, const void* q, const void* g,
+                               const sana_rope* rope, const float* S, const float* z, float eps,
+                               void* out, sana_stream_t stream) {
+  const char* who = "sana_linattn_apply";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!q || !S || !z || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!std::isfinite(eps) || eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", who);
+  const void* ptrs[5] = {q, g, S, z, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
+  const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
+  if (overlap(out, n, q, n) || overlap(out, n, g, n) || overlap(out, n, S, sb))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an input", who);
+  return linattn_apply_run(*s, dt, q, g, to_dev(*rope), S, z, eps, out, stream);
+}
+
+size_t sana_softmax_anchor_workspace_size(const sana_shape* s, sana_dtype dt) {
+  if (check_shape(s, dt, "sana_softmax_anchor_workspace_size") != SANA_OK) return 0;
+  return anchor_ws_bytes(*s, dt);
+}
+
+sana_status sana_softmax_anchor_fwd(const sana_shape* s, sana_dtype dt, const void* q,
+                                    const void* k, const void* v, const void* g,
+                                    const sana_rope* rope, float scale, void* out, void* ws,
+                                    size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_softmax_anchor_fwd";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (rope)
+    if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  if (!std::isfinite(scale)) return fail(SANA_ERR_INVALID_ARG, "%s: scale is not finite", who);
+  const void* ptrs[5] = {q, k, v, g, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
+  if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, g, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an input", who);
+  const size_t need = anchor_ws_bytes(*s, dt);
+  if (need && (!ws || ws_bytes < need))
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  RopeDev rd{};
+  if (rope) rd = to_dev(*rope);
+  return anchor_run(*s, dt, q, k, v, g, rope ? &rd : nullptr, scale, out, ws, ws_bytes, stream);
+}
+
+sana_status sana_attnres_route(int B, long long N, int C, sana_dtype dt, const void* const* sources,
+                               int num_sources, const float* w, float rms_eps, void* h_out,
+                               float* alpha_out, sana_stream_t stream) {
+  const char* who = "sana_attnres_route";
+  if (dt != SANA_F32 && dt != SANA_BF16) return fail(SANA_ERR_INVALID_ARG, "%s: bad dtype", who);
+  if (B < 1 || N < 0 || C < 1) return fail(SANA_ERR_INVALID_ARG, "%s: bad sizes", who);
+  if (!sources || !w || !h_out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (num_sources < 1 || num_sources > 16)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: num_sources=%d (1..16)", who, num_sources);
+  if (!std::isfinite(rms_eps) || rms_eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: bad rms_eps", who);
+  const size_t n = (size_t)B * N * C * esize(dt);
+  for (int i = 0; i < num_sources; ++i) {
+    if (!sources[i] || !aligned16(sources[i]))
+      return fail(SANA_ERR_INVALID_ARG, "%s: source %d is NULL or not 16-byte aligned", who, i);
+    if (overlap(h_out, n, sources[i], n)) return fail(SANA_ERR_INVALID_ARG, "%s: h_out aliases source %d", who, i);
+  }
+  if (!aligned16(h_out) || !aligned16(w)) return fail(SANA_ERR_INVALID_ARG, "%s: h_out / w not 16-byte aligned", who);
+  return attnres_run(B, N, C, dt, sources, num_sources, w, rms_eps, h_out, alpha_out, false,
+                     nullptr, stream);
+}
+
+sana_status sana_rmsnorm(long long rows, int C, sana_dtype dt, const void* x, float eps, void* y,
+                         sana_stream_t stream) {
+  if (dt != SANA_F32 && dt != SANA_BF16) return fail(SANA_ERR_INVALID_ARG, "sana_rmsnorm: bad dtype");
+  if (rows < 0 || C < 1 || !x || !y) return fail(SANA_ERR_INVALID_ARG, "sana_rmsnorm: bad arguments");
+  if (!aligned16(x) || !aligned16(y)) return fail(SANA_ERR_INVALID_ARG, "sana_rmsnorm: pointers not 16-byte aligned");
+  return rmsnorm_run(rows, C, dt, x, eps, y, stream);
+}
+
+sana_status sana_gemm_bf16(long long M, int N, int K, const void* A, long long lda, const void* W,
+                           void* out, long long ldo, int epilogue, sana_stream_t stream) {
+  const char* who = "sana_gemm_bf16";
+  if (M < 0 || N < 1 || K < 1 || !A || !W || !out) return fail(SANA_ERR_INVALID_ARG, "%s: bad arguments", who);
+  if (K % 64 != 0 || N % 8 != 0 || lda < K || ldo < N || lda % 8 || ldo % 8)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: needs K %% 64 == 0, N %% 8 == 0, lda >= K, ldo >= N (multiples of 8)", who);
+  if (epilogue < 0 || epilogue > 2) return fail(SANA_ERR_INVALID_ARG, "%s: bad epilogue %d", who, epilogue);
+  if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers not 16-byte aligned", who);
+  return gemm_run(M, N, K, A, lda, W, out, ldo, epilogue, stream);
+}
+
+sana_status sana_sync_status(sana_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(SANA_ERR_CUDA, "sana_sync_status: %s", cudaGetErrorString(e));
+  int* sw = status_word();
+  if (!sw) return fail(SANA_ERR_CUDA, "sana_sync_status: no status word on this device");
+  int v = 0;
+  e = cudaMemcpy(&v, sw, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(SANA_ERR_CUDA, "sana_sync_status: %s", cudaGetErrorString(e));
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(sw, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(SANA_ERR_TIMEOUT, "a kernel gave up a bounded wait (code 0x%x)", v);
+  }
+  return SANA_OK;
+}
+
+}  // extern "C"

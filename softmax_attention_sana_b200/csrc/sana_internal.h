@@ -1,0 +1,111 @@
+// Host-side internals of libsana: error reporting, TMA tensor-map encoding,
+// workspace carving and the launchers each entry point dispatches to.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/sana.h"
+
+namespace sana {
+
+// Fixed SM count of the target part.  Work partitions (and therefore the
+// summation order of split reductions) depend only on the problem shape.
+constexpr int kNumSMs = 148;
+
+sana_status fail(sana_status st, const char* fmt, ...);
+sana_status check_launch(const char* what);
+// Device address of the status word of the current device.
+int* status_word();
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over a caller-provided workspace.
+struct Carver {
+  char* base;
+  size_t cap;
+  size_t used = 0;
+  Carver(void* b, size_t c) : base(static_cast<char*>(b)), cap(c) {}
+  template <class T>
+  T* take(size_t count) {
+    used = align_up(used, 256);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+  bool fits() const { return used <= cap; }
+};
+
+// TMA descriptors (bf16, 128-byte swizzle, zero fill out of bounds).
+// 3D view of a (B, rows, cols) tensor with a row stride of `row_stride` elements
+// and a batch stride of `batch_stride` elements; box = (64 cols, box_rows rows, 1).
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                       uint64_t batches, uint64_t row_stride, uint64_t batch_stride,
+                       uint32_t box_rows);
+// 2D view of a (rows, cols) tensor with row stride `row_stride` elements.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                       uint64_t row_stride, uint32_t box_cols, uint32_t box_rows);
+
+// Grid of one call, as the kernels see it.
+struct GridDev {
+  int T, H, W;
+  int t_offset;
+  int N;
+  int heads;
+};
+// RoPE tables, as the kernels see them.
+struct RopeDev {
+  const float *cos_t, *sin_t, *cos_h, *sin_h, *cos_w, *sin_w;
+  int n_t, n_h, n_w;
+};
+
+inline int odd_up(int n) { return n | 1; }
+inline size_t rope_smem_bytes(const GridDev& g, const RopeDev& r) {
+  return 8 * ((size_t)g.T * odd_up(r.n_t) + (size_t)g.H * odd_up(r.n_h) +
+              (size_t)g.W * odd_up(r.n_w));
+}
+// The tcgen05 kernels stage the rotary tables of one grid in shared memory.
+constexpr size_t kRopeSmemMax = 26 * 1024;
+
+// ---------------------------------------------------------------- linear attention
+struct LinAttnPlan {
+  int splits_a;  // CTAs per (batch, head) of the state reduction
+  int splits_b;  // CTAs per (batch, head) of the output pass
+  int tiles;     // 128-token tiles per (batch, head)
+};
+LinAttnPlan linattn_plan(const sana_shape& s, sana_dtype dt);
+size_t linattn_ws_bytes(const sana_shape& s, sana_dtype dt);
+size_t linattn_state_ws_bytes(const sana_shape& s, sana_dtype dt);
+sana_status linattn_state_run(const sana_shape& s, sana_dtype dt, const void* k, const void* v,
+                              const RopeDev& rope, float* S_out, float* z_out, void* ws,
+                              size_t ws_bytes, cudaStream_t st);
+sana_status linattn_apply_run(const sana_shape& s, sana_dtype dt, const void* q, const void* gt,
+                              const RopeDev& rope, const float* S, const float* z, float eps,
+                              void* out, cudaStream_t st);
+
+// Bidirectional (S_prev == nullptr) or block-causal step.
+sana_status linattn_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,
+                        const void* v, const void* g, const RopeDev& rope, float eps,
+                        float* state_S, float* state_z, bool causal, bool commit, void* out,
+                        void* ws, size_t ws_bytes, cudaStream_t st);
+
+// ---------------------------------------------------------------- softmax anchor
+size_t anchor_ws_bytes(const sana_shape& s, sana_dtype dt);
+sana_status anchor_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,
+                       const void* v, const void* g, const RopeDev* rope, float scale,
+                       void* out, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// ---------------------------------------------------------------- AttnRes / norm / GEMM
+sana_status attnres_run(int B, long long N, int C, sana_dtype dt, const void* const* sources,
+                        int S, const float* w, float eps, void* h, float* alpha, bool normed_out,
+                        void* h_norm, cudaStream_t st);
+sana_status rmsnorm_run(long long rows, int C, sana_dtype dt, const void* x, float eps, void* y,
+                        cudaStream_t st);
+sana_status gemm_run(long long M, int N, int K, const void* A, long long lda, const void* W,
+                     void* out, long long ldo, int epilogue, cudaStream_t st);
+
+}  // namespace sana

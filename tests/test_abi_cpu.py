@@ -1,0 +1,122 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol
+include/sana.h declares, computes the RoPE tables on the host like the oracle,
+and rejects bad arguments before touching the device."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from tests._sana import _lib, sana
+from oracle import sana_oracle as orc
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sana.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sana_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_error_string():
+    assert b"sm_100a" in _lib.lib.sana_version()
+    assert isinstance(_lib.last_error(), str)
+
+
+@pytest.mark.parametrize("grid,split,t_total", [((2, 4, 4), (2, 3, 3), 2), ((21, 45, 80), (22, 21, 21), 21),
+                                                ((3, 45, 80), (22, 21, 21), 241)])
+def test_host_rope_tables_match_oracle_angles(grid, split, t_total):
+    T, H, W = grid
+    tab = _lib.host_rope_tables(t_total, H, W, split).numpy().astype(np.float64)
+    n_t, n_h, n_w = split
+    off = 0
+    parts = {}
+    for name, npos, npair in (("t", t_total, n_t), ("h", H, n_h), ("w", W, n_w)):
+        c = tab[off:off + npos * npair].reshape(npos, npair)
+        s = tab[off + npos * npair:off + 2 * npos * npair].reshape(npos, npair)
+        parts[name] = (c, s)
+        off += 2 * npos * npair
+    # oracle angles for the frames [t0, t0 + T)
+    t0 = t_total - T
+    ang = orc.rope_angles(T, H, W, *split, t_offset=t0)
+    t, h, w = orc.token_grid(T, H, W, t0)
+    got_c = np.concatenate([parts["t"][0][t], parts["h"][0][h], parts["w"][0][w]], axis=1)
+    got_s = np.concatenate([parts["t"][1][t], parts["h"][1][h], parts["w"][1][w]], axis=1)
+    # fp32 rounding of cos / sin evaluated in double
+    assert np.max(np.abs(got_c - np.cos(ang))) < 1e-7
+    assert np.max(np.abs(got_s - np.sin(ang))) < 1e-7
+
+
+def _shape(**kw):
+    d = dict(B=1, T=2, H=4, W=4, heads=2, head_dim=16, t_offset=0)
+    d.update(kw)
+    return _lib.Shape(d["B"], d["T"], d["H"], d["W"], d["heads"], d["head_dim"], d["t_offset"])
+
+
+def test_workspace_sizes():
+    L = _lib.lib
+    assert L.sana_linattn_workspace_size(ctypes.byref(_shape()), _lib.SANA_F32) > 0
+    s720 = _shape(T=21, H=45, W=80, heads=24, head_dim=128)
+    ws = L.sana_linattn_workspace_size(ctypes.byref(s720), _lib.SANA_BF16)
+    # 6 splits x 24 heads of (128x128 + 128) fp32 partials, S^T in bf16, z: about 10 MB
+    assert 9e6 < ws < 12e6
+    assert L.sana_softmax_anchor_workspace_size(ctypes.byref(s720), _lib.SANA_BF16) >= 2 * 75600 * 3072 * 2
+    # unsupported shapes report 0
+    assert L.sana_linattn_workspace_size(ctypes.byref(_shape(head_dim=64)), _lib.SANA_BF16) == 0
+
+
+def _call_fwd(shape, dtype, ptr=16, rope=None, eps=1e-6, ws_bytes=1 << 20):
+    r = rope or _lib.RopeStruct(16, 16, 16, 16, 16, 16, 2, 3, 3, 2, 4, 4)
+    return _lib.lib.sana_linattn_fwd(ctypes.byref(shape) if shape is not None else None, dtype,
+                                     ptr, ptr + 4096, ptr + 8192, None, ctypes.byref(r), eps,
+                                     ptr + 16384, 1 << 20, ws_bytes, None)
+
+
+def test_validation_errors_return_before_any_device_work():
+    L = _lib
+    # NULL shape
+    assert _call_fwd(None, L.SANA_F32) == L.SANA_ERR_INVALID_ARG
+    # bf16 requires head_dim 128
+    assert _call_fwd(_shape(head_dim=16), L.SANA_BF16) == L.SANA_ERR_UNSUPPORTED
+    assert "head_dim" in L.last_error()
+    # fp32 head_dim outside {16, 32, 64, 128}
+    assert _call_fwd(_shape(head_dim=24), L.SANA_F32) == L.SANA_ERR_UNSUPPORTED
+    # rope split not covering head_dim / 2
+    bad = _lib.RopeStruct(16, 16, 16, 16, 16, 16, 2, 3, 2, 2, 4, 4)
+    assert _call_fwd(_shape(), L.SANA_F32, rope=bad) == L.SANA_ERR_INVALID_ARG
+    # tables that do not cover the frames
+    short = _lib.RopeStruct(16, 16, 16, 16, 16, 16, 2, 3, 3, 1, 4, 4)
+    assert _call_fwd(_shape(), L.SANA_F32, rope=short) == L.SANA_ERR_INVALID_ARG
+    # misaligned pointer
+    assert _call_fwd(_shape(), L.SANA_F32, ptr=18) == L.SANA_ERR_INVALID_ARG
+    # negative eps
+    assert _call_fwd(_shape(), L.SANA_F32, eps=-1.0) == L.SANA_ERR_INVALID_ARG
+    # workspace too small
+    assert _call_fwd(_shape(), L.SANA_F32, ws_bytes=16) == L.SANA_ERR_WORKSPACE
+    # output aliasing an input
+    r = _lib.RopeStruct(16, 16, 16, 16, 16, 16, 2, 3, 3, 2, 4, 4)
+    st = L.lib.sana_linattn_fwd(ctypes.byref(_shape()), L.SANA_F32, 4096, 8192, 12288, None,
+                                ctypes.byref(r), 1e-6, 4096, 1 << 20, 1 << 20, None)
+    assert st == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
+
+
+def test_attnres_and_gemm_validation():
+    L = _lib
+    arr = (ctypes.c_void_p * 1)(4096)
+    assert L.lib.sana_attnres_route(1, 10, 64, L.SANA_BF16, arr, 0, 8192, 1e-6, 16384, None, None) \
+        == L.SANA_ERR_UNSUPPORTED
+    assert L.lib.sana_attnres_route(1, 10, 60, L.SANA_BF16, arr, 1, 8192, 1e-6, 1 << 20, None, None) \
+        == L.SANA_ERR_UNSUPPORTED
+    assert L.lib.sana_gemm_bf16(128, 128, 100, 4096, 100, 8192, 1 << 20, 128, 0, None) \
+        == L.SANA_ERR_UNSUPPORTED
