@@ -412,8 +412,9 @@ static sana_status linattn_common(const char* who, const sana_shape* s, sana_dty
                                   sana_stream_t stream) {
   if (sana_status e = check_shape(s, dt, who)) return e;
   if (sana_status e = check_rope(rope, s, who)) return e;
-  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
   if (!std::isfinite(eps) || eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", who);
+  if (s->T == 0) return SANA_OK;  // empty grid: nothing to read or write, state unchanged
+  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
   const void* ptrs[5] = {q, k, v, g, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
@@ -464,10 +465,11 @@ sana_status sana_linattn_state(const sana_shape* s, sana_dtype dt, const void* k
   const char* who = "sana_linattn_state";
   if (sana_status e = check_shape(s, dt, who)) return e;
   if (sana_status e = check_rope(rope, s, who)) return e;
-  if (!k || !v || !S_out || !z_out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!S_out || !z_out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL state pointer", who);
+  if (s->T > 0 && (!k || !v)) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
   const void* ptrs[4] = {k, v, S_out, z_out};
   for (const void* p : ptrs)
-    if (!aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
   const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
   const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
   const size_t zb = (size_t)s->B * s->heads * s->head_dim * 4;
@@ -488,8 +490,9 @@ sana_status sana_linattn_apply(const sana_shape* s, sana_dtype dt, const void* q
   const char* who = "sana_linattn_apply";
   if (sana_status e = check_shape(s, dt, who)) return e;
   if (sana_status e = check_rope(rope, s, who)) return e;
-  if (!q || !S || !z || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
   if (!std::isfinite(eps) || eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", who);
+  if (s->T == 0) return SANA_OK;
+  if (!q || !S || !z || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
   const void* ptrs[5] = {q, g, S, z, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
@@ -513,8 +516,9 @@ sana_status sana_softmax_anchor_fwd(const sana_shape* s, sana_dtype dt, const vo
   if (sana_status e = check_shape(s, dt, who)) return e;
   if (rope)
     if (sana_status e = check_rope(rope, s, who)) return e;
-  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
   if (!std::isfinite(scale)) return fail(SANA_ERR_INVALID_ARG, "%s: scale is not finite", who);
+  if (s->T == 0) return SANA_OK;
+  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
   const void* ptrs[5] = {q, k, v, g, out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
@@ -537,6 +541,9 @@ sana_status sana_attnres_route(int B, long long N, int C, sana_dtype dt, const v
   const char* who = "sana_attnres_route";
   if (dt != SANA_F32 && dt != SANA_BF16) return fail(SANA_ERR_INVALID_ARG, "%s: bad dtype", who);
   if (B < 1 || N < 0 || C < 1) return fail(SANA_ERR_INVALID_ARG, "%s: bad sizes", who);
+  if (num_sources < 1 || num_sources > 16)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: num_sources=%d (1..16)", who, num_sources);
+  if (N == 0) return SANA_OK;
   if (!sources || !w || !h_out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
   if (num_sources < 1 || num_sources > 16)
     return fail(SANA_ERR_UNSUPPORTED, "%s: num_sources=%d (1..16)", who, num_sources);

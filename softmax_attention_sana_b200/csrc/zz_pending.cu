@@ -1,6 +1,5 @@
 #include "sana_internal.h"
 namespace sana {
-sana_status anchor_bf16_run(const sana_shape&, const void*, const void*, const void*, const void*, const GridDev&, void*, cudaStream_t) { return fail(SANA_ERR_UNSUPPORTED, "bf16 anchor: not built yet"); }
 sana_status gemm_run(long long, int, int, const void*, long long, const void*, void*, long long, int, cudaStream_t) { return fail(SANA_ERR_UNSUPPORTED, "gemm: not built yet"); }
 }
 extern "C" size_t sana_hybrid_stack_workspace_size(const sana_shape*, const sana_stack_config*) { return 0; }

@@ -1,0 +1,98 @@
+"""GPU parity of the gated softmax anchor against the float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import sana_inputs as si
+from oracle import sana_oracle as orc
+from tests._sana import sana
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-4
+BF16_TOL = 2e-2
+
+
+def f64(t):
+    return si.as_f64(t)
+
+
+def gpu_anchor(q, k, v, g, grid, split, heads, use_rope=True):
+    rope = sana.Rope(grid[0], grid[1], grid[2], split) if use_rope else None
+    y = sana.softmax_anchor_fwd(q.cuda(), k.cuda(), v.cuda(), None if g is None else g.cuda(),
+                                rope, grid, heads)
+    sana.sync_status()
+    return y.cpu()
+
+
+def test_tiny_fp32_config():
+    wl = si.TINY
+    q, k, v, g = si.qkvg(wl)
+    grid = (wl.T, wl.H, wl.W)
+    y = gpu_anchor(q, k, v, g, grid, wl.rope_split, wl.heads)
+    yo = orc.softmax_anchor(f64(q), f64(k), f64(v), grid, wl.rope_split, wl.heads, gate=f64(g))
+    assert orc.max_rel_err(f64(y), yo) <= F32_TOL
+    y = gpu_anchor(q, k, v, None, grid, wl.rope_split, wl.heads, use_rope=False)
+    yo = orc.softmax_anchor(f64(q), f64(k), f64(v), None, None, wl.heads, use_rope=False)
+    assert orc.max_rel_err(f64(y), yo) <= F32_TOL
+
+
+@pytest.mark.parametrize("B,heads,grid", [(1, 2, (2, 4, 4)),      # N = 32: one partial tile
+                                          (2, 3, (3, 5, 9)),      # N = 135: ragged key/query tail
+                                          (1, 1, (1, 1, 1)),      # a single key
+                                          (1, 2, (5, 16, 16)),    # N = 1280: 10 full tiles
+                                          (1, 2, (7, 13, 17))])   # N = 1547
+def test_bf16_small_with_ragged_tails(B, heads, grid):
+    N = grid[0] * grid[1] * grid[2]
+    C = heads * 128
+    q, k, v, g = (si.normal(11000 + 10 * N + i, (B, N, C)) for i in range(4))
+    split = (22, 21, 21)
+    y = gpu_anchor(q, k, v, g, grid, split, heads)
+    yo = orc.softmax_anchor(f64(q), f64(k), f64(v), grid, split, heads, gate=f64(g))
+    assert orc.max_rel_err(f64(y), yo) <= BF16_TOL
+    y = gpu_anchor(q, k, v, None, grid, split, heads, use_rope=False)
+    yo = orc.softmax_anchor(f64(q), f64(k), f64(v), None, None, heads, use_rope=False)
+    assert orc.max_rel_err(f64(y), yo) <= BF16_TOL
+
+
+def test_bf16_large_logits_exercise_rescaling():
+    """Q scaled up so the running max jumps by far more than the lazy-rescale
+    threshold across key tiles."""
+    grid, heads = (4, 8, 16), 2
+    N = 512
+    q = si.normal(11500, (1, N, 256), scale=6.0)
+    k, v, g = (si.normal(11501 + i, (1, N, 256)) for i in range(3))
+    # make later key tiles dominate for some queries
+    k[:, 384:] *= 3
+    split = (22, 21, 21)
+    y = gpu_anchor(q, k, v, g, grid, split, heads)
+    yo = orc.softmax_anchor(f64(q), f64(k), f64(v), grid, split, heads, gate=f64(g))
+    assert orc.max_rel_err(f64(y), yo) <= BF16_TOL
+
+
+def test_720p_full_size_sampled_rows():
+    """720p/5s anchor layer: 192 seeded query rows per head (plus the ragged
+    tail) against the oracle over all 75,600 keys; bit-reproducible."""
+    wl = si.P720
+    q, k, v, g = si.qkvg(wl)
+    grid = (wl.T, wl.H, wl.W)
+    rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
+    args = [t.cuda() for t in (q, k, v, g)]
+    y = sana.softmax_anchor_fwd(*args, rope, grid, wl.heads)
+    y2 = sana.softmax_anchor_fwd(*args, rope, grid, wl.heads)
+    sana.sync_status()
+    assert torch.equal(y, y2)
+    y = y.cpu()
+    rng = np.random.default_rng(33)
+    rows = np.unique(np.concatenate([rng.choice(wl.N, 192, replace=False),
+                                     np.arange(wl.N - 16, wl.N)]))
+    D = wl.D
+    got, ref = [], []
+    for h in range(wl.heads):
+        sl = slice(h * D, (h + 1) * D)
+        ref.append(orc.softmax_anchor(f64(q[:, :, sl]), f64(k[:, :, sl]), f64(v[:, :, sl]), grid,
+                                      wl.rope_split, 1, gate=f64(g[:, :, sl]), rows=rows))
+        got.append(f64(y[:, rows, sl]))
+    err = orc.max_rel_err(np.concatenate(got, -1), np.concatenate(ref, -1))
+    assert err <= BF16_TOL, err
