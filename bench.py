@@ -294,6 +294,9 @@ def components(sana, args):
     out["attnres_route_720p_3src"] = {"ms": ms, "GB_per_s": 4 * TENSOR_BYTES / (ms / 1e3) / 1e9}
     del srcs, h
     # softmax anchor at 720p/5s
+    if args.no_anchor:
+        out["softmax_anchor_720p"] = {"skipped": "--no-anchor"}
+        return out
     try:
         q, k, v, g = (t.cuda() for t in si.qkvg(WL))
         rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
@@ -418,6 +421,7 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=150.0,
                     help="seconds the --impl reference run aims to take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-anchor", action="store_true", help="leave the anchor out of the components")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -71,7 +71,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
                     errors.append(src)
     if errors:
         raise RuntimeError("nvcc failed for: " + ", ".join(os.path.basename(e) for e in errors))
-    if force or jobs or not os.path.exists(LIB):
+    stale = not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs)
+    if force or jobs or stale:
         cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
                *objs, "-o", LIB + ".tmp"]
         p = subprocess.run(cmd, capture_output=True, text=True)

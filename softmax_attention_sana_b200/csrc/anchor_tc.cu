@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; ok && j < nkv; ++j) {
       const int bb = j & 1;
-      if (!mbar_wait(&ctl.s_full[bb], (j >> 1) & 1, wc, 0x38)) {
+      // warp-uniform outcome: tcgen05.ld / st are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl.s_full[bb], (j >> 1) & 1, wc, 0x38))) {
         ok = false;
         break;
       }
@@ -208,11 +209,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx = fmaxf(mx, s);
         }
       const float m_new = fmaxf(m, mx);
-      if (m_new > m + kRescaleLog2) {
-        const float corr = ex2(m - m_new);  // 0 on the first tile
+      // rescale O when any row of the warp needs it (collective TMEM access)
+      const bool grow = m_new > m + kRescaleLog2;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float m_use = grow ? m_new : m;
+        const float corr = ex2(m - m_use);  // 0 on the first tile, 1 for rows that keep m
         if (j >= 1) {
-          // O holds sum over tiles < j; wait for the last PV before touching it
-          if (!mbar_wait(&ctl.pv_done, (j - 1) & 1, wc, 0x39)) {
+          // O holds the sum over tiles < j; wait for the last PV before touching it
+          if (!__all_sync(0xffffffffu, mbar_wait(&ctl.pv_done, (j - 1) & 1, wc, 0x39))) {
             ok = false;
             break;
           }
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st_wait();
         }
         l *= corr;
-        m = m_new;
+        m = m_use;
       }
       float rs = 0.f;
       uint32_t pk[2][32];
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&ctl.p_full[bb]);
     }
     // ---------------- epilogue: Y = O / l * sigmoid(G)
-    ok = ok && nkv > 0 && mbar_wait(&ctl.pv_done, (nkv - 1) & 1, wc, 0x3a);
+    ok = __all_sync(0xffffffffu, ok && nkv > 0 && mbar_wait(&ctl.pv_done, (nkv - 1) & 1, wc, 0x3a));
     uint8_t* ybuf = kGate ? g_s : q_s;
     if (ok) {
       tc_fence_after();

@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       fence_proxy_async_smem();
       mbar_arrive(&ctl.kready[s]);
     }
-    const bool ok = mbar_wait(&ctl.done, 0, wc, 0x14);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl.done, 0, wc, 0x14));
     tc_fence_after();
     const size_t part = ((size_t)(b * g.heads + h) * splits + split);
     if (ok) {
@@ -418,6 +418,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       // both column halves have written their partial denominators
       mbar_arrive(&ctl.wsync);
       okw = mbar_wait(&ctl.wsync, (n_wsync++) & 1, wc, 0x29) && okw;
+      okw = __all_sync(0xffffffffu, okw);  // tcgen05.ld is warp-collective
       const float inv = 1.f / (ctl.den[s][0][r] + ctl.den[s][1][r] + eps);
       uint32_t acc[2][32];
       if (okw) {

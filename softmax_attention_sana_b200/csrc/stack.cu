@@ -1,0 +1,180 @@
+// Hybrid linear-softmax stack forward: the host-side schedule over the
+// kernels, all launches stream-ordered with no host synchronisation.
+//
+//   "SANA-Video 2.0" abstract: three gated linear-attention layers to one
+//   gated softmax anchor (3:1).  hyper.ai summary, Method: Block Attention
+//   Residuals -- sublayer outputs accumulate into a running partial sum, a
+//   completed block of `block_span` layers freezes it as a block summary, and
+//   every sublayer reads h = sum_i softmax_i(w . RMSNorm(v_i)) v_i over
+//   [embedding, block summaries, partial sum] with one shared query for the
+//   attention sublayers and one for the FFN sublayers.
+//
+// Per layer (AttnRes on):
+//   route(w_attn) + RMSNorm  -> x_hat            (one fused kernel)
+//   x_hat . W_qkvg^T         -> Q, K, V, G       (one GEMM, output split in 4)
+//   linear attention | softmax anchor -> a
+//   a . W_o^T                -> partial (+)=     (GEMM, residual epilogue)
+//   route(w_ffn) + RMSNorm   -> x_hat
+//   SiLU(x_hat . W_up^T)     -> u                (GEMM, SiLU epilogue)
+//   u . W_down^T             -> partial +=       (GEMM, residual epilogue)
+//   every block_span layers: partial becomes a summary (pointer hand-over).
+#include <cmath>
+#include <vector>
+
+#include "sana_common.cuh"
+#include "sana_internal.h"
+
+namespace sana {
+
+sana_status gemm_run_parts(long long M, int N, int K, const void* A, long long lda, const void* W,
+                           void* const* outs, int nparts, long long ldo, int epilogue,
+                           cudaStream_t st);
+
+namespace {
+
+struct StackWs {
+  __nv_bfloat16 *xhat, *q, *k, *v, *g, *attn, *ffn;
+  std::vector<__nv_bfloat16*> blocks;  // summaries + the running partial sum
+  void* attn_ws;
+  size_t attn_ws_bytes;
+  size_t bytes;
+};
+
+StackWs carve_stack(const sana_shape& s, const sana_stack_config& c, void* ws) {
+  const size_t tok = (size_t)s.B * s.T * s.H * s.W;
+  const size_t C = (size_t)s.heads * s.head_dim;
+  Carver cv(ws, ~size_t(0));
+  StackWs w{};
+  w.xhat = cv.take<__nv_bfloat16>(tok * C);
+  w.q = cv.take<__nv_bfloat16>(tok * C);
+  w.k = cv.take<__nv_bfloat16>(tok * C);
+  w.v = cv.take<__nv_bfloat16>(tok * C);
+  w.g = cv.take<__nv_bfloat16>(tok * C);
+  w.attn = cv.take<__nv_bfloat16>(tok * C);
+  w.ffn = c.ffn_mult > 0 ? cv.take<__nv_bfloat16>(tok * C * c.ffn_mult) : nullptr;
+  if (c.use_attnres) {
+    const int nblocks = (c.layers + c.block_span - 1) / c.block_span;
+    for (int i = 0; i < nblocks; ++i) w.blocks.push_back(cv.take<__nv_bfloat16>(tok * C));
+  }
+  const size_t lin = linattn_ws_bytes(s, SANA_BF16), anc = anchor_ws_bytes(s, SANA_BF16);
+  w.attn_ws_bytes = lin > anc ? lin : anc;
+  w.attn_ws = cv.take<char>(w.attn_ws_bytes);
+  w.bytes = align_up(cv.used, 256);
+  return w;
+}
+
+sana_status check_cfg(const sana_shape* s, const sana_stack_config* c) {
+  if (!s || !c) return fail(SANA_ERR_INVALID_ARG, "stack: NULL shape or config");
+  if (s->head_dim != 128) return fail(SANA_ERR_UNSUPPORTED, "stack: bf16 path needs head_dim 128");
+  if (s->B < 1 || s->T < 1 || s->H < 1 || s->W < 1 || s->heads < 1)
+    return fail(SANA_ERR_INVALID_ARG, "stack: bad shape");
+  if (s->heads * 128 % 256 != 0)
+    return fail(SANA_ERR_UNSUPPORTED, "stack: hidden size must be a multiple of 256");
+  if (c->layers < 1 || c->ratio < 1 || c->ffn_mult < 0 || c->ffn_mult > 8 ||
+      (c->use_attnres && c->block_span < 1))
+    return fail(SANA_ERR_INVALID_ARG, "stack: bad config");
+  if (c->use_attnres && 1 + (c->layers + c->block_span - 1) / c->block_span > 16)
+    return fail(SANA_ERR_UNSUPPORTED, "stack: more than 16 AttnRes sources");
+  if (!(c->eps >= 0.f) || !(c->rms_eps >= 0.f)) return fail(SANA_ERR_INVALID_ARG, "stack: bad eps");
+  return SANA_OK;
+}
+
+}  // namespace
+}  // namespace sana
+
+using namespace sana;
+
+extern "C" size_t sana_hybrid_stack_workspace_size(const sana_shape* s, const sana_stack_config* c) {
+  if (check_cfg(s, c) != SANA_OK) return 0;
+  return carve_stack(*s, *c, nullptr).bytes;
+}
+
+extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_stack_config* c,
+                                             const sana_stack_weights* w, const sana_rope* rope,
+                                             const void* x_embed, void* out, void* ws,
+                                             size_t ws_bytes, sana_stream_t st) {
+  if (sana_status e = check_cfg(s, c)) return e;
+  if (!w || !rope || !x_embed || !out || !w->w_qkvg || !w->w_o)
+    return fail(SANA_ERR_INVALID_ARG, "stack: NULL argument");
+  if (c->ffn_mult > 0 && (!w->w_up || !w->w_down))
+    return fail(SANA_ERR_INVALID_ARG, "stack: FFN weights are NULL");
+  if (c->use_attnres && (!w->w_attn || (c->ffn_mult > 0 && !w->w_ffn)))
+    return fail(SANA_ERR_INVALID_ARG, "stack: router queries are NULL");
+  if (rope->n_t + rope->n_h + rope->n_w != 64 || rope->H != s->H || rope->W != s->W ||
+      rope->T_total < s->t_offset + s->T)
+    return fail(SANA_ERR_INVALID_ARG, "stack: rope tables do not match the grid");
+  const size_t need = carve_stack(*s, *c, nullptr).bytes;
+  if (!ws || ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "stack: workspace %zu < %zu bytes", ws ? ws_bytes : 0, need);
+  const StackWs P = carve_stack(*s, *c, ws);
+  const int C = s->heads * 128, F = c->ffn_mult * C;
+  const long long M = (long long)s->B * s->T * s->H * s->W;
+  const long long Nseq = (long long)s->T * s->H * s->W;
+  const RopeDev rd{rope->cos_t, rope->sin_t, rope->cos_h, rope->sin_h, rope->cos_w, rope->sin_w,
+                   rope->n_t, rope->n_h, rope->n_w};
+  const float scale = c->anchor_scale > 0.f ? c->anchor_scale : 1.f / sqrtf(128.f);
+  auto attention = [&](int l) -> sana_status {
+    void* parts[4] = {P.q, P.k, P.v, P.g};
+    if (sana_status e = gemm_run_parts(M, 4 * C, C, P.xhat, C, w->w_qkvg[l], parts, 4, C, 0, st))
+      return e;
+    if (l % c->ratio == c->ratio - 1)
+      return anchor_run(*s, SANA_BF16, P.q, P.k, P.v, P.g, &rd, scale, P.attn, P.attn_ws,
+                        P.attn_ws_bytes, st);
+    return linattn_run(*s, SANA_BF16, P.q, P.k, P.v, P.g, rd, c->eps, nullptr, nullptr, false,
+                       false, P.attn, P.attn_ws, P.attn_ws_bytes, st);
+  };
+
+  if (!c->use_attnres) {
+    // plain pre-norm residual stream in `out`
+    if (cudaMemcpyAsync(out, x_embed, (size_t)M * C * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return fail(SANA_ERR_CUDA, "stack: copy of the embedding failed");
+    for (int l = 0; l < c->layers; ++l) {
+      if (sana_status e = rmsnorm_run(M, C, SANA_BF16, out, c->rms_eps, P.xhat, st)) return e;
+      if (sana_status e = attention(l)) return e;
+      if (sana_status e = gemm_run(M, C, C, P.attn, C, w->w_o[l], out, C, 2, st)) return e;
+      if (c->ffn_mult > 0) {
+        if (sana_status e = rmsnorm_run(M, C, SANA_BF16, out, c->rms_eps, P.xhat, st)) return e;
+        if (sana_status e = gemm_run(M, F, C, P.xhat, C, w->w_up[l], P.ffn, F, 1, st)) return e;
+        if (sana_status e = gemm_run(M, C, F, P.ffn, F, w->w_down[l], out, C, 2, st)) return e;
+      }
+    }
+    return SANA_OK;
+  }
+
+  // AttnRes: sources = [embedding, summaries..., partial (when non-empty)]
+  std::vector<const void*> src;
+  int nsum = 0;
+  bool partial_live = false;
+  auto sources = [&]() {
+    src.clear();
+    src.push_back(x_embed);
+    for (int i = 0; i < nsum; ++i) src.push_back(P.blocks[i]);
+    if (partial_live) src.push_back(P.blocks[nsum]);
+  };
+  for (int l = 0; l < c->layers; ++l) {
+    __nv_bfloat16* partial = P.blocks[nsum];
+    sources();
+    if (sana_status e = attnres_run(s->B, Nseq, C, SANA_BF16, src.data(), (int)src.size(),
+                                    w->w_attn, c->rms_eps, nullptr, nullptr, true, P.xhat, st))
+      return e;
+    if (sana_status e = attention(l)) return e;
+    if (sana_status e = gemm_run(M, C, C, P.attn, C, w->w_o[l], partial, C, partial_live ? 2 : 0, st))
+      return e;
+    partial_live = true;
+    if (c->ffn_mult > 0) {
+      sources();
+      if (sana_status e = attnres_run(s->B, Nseq, C, SANA_BF16, src.data(), (int)src.size(),
+                                      w->w_ffn, c->rms_eps, nullptr, nullptr, true, P.xhat, st))
+        return e;
+      if (sana_status e = gemm_run(M, F, C, P.xhat, C, w->w_up[l], P.ffn, F, 1, st)) return e;
+      if (sana_status e = gemm_run(M, C, F, P.ffn, F, w->w_down[l], partial, C, 2, st)) return e;
+    }
+    if ((l + 1) % c->block_span == 0) {  // freeze the block summary
+      ++nsum;
+      partial_live = false;
+    }
+  }
+  sources();
+  return attnres_run(s->B, Nseq, C, SANA_BF16, src.data(), (int)src.size(), w->w_attn,
+                     c->rms_eps, out, nullptr, false, nullptr, st);
+}
