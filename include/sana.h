@@ -236,6 +236,24 @@ SANA_API sana_status sana_hybrid_stack_fwd(const sana_shape* shape, const sana_s
                                   sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Allocation-free linear attention (the pages have no counterpart; this is a
+ * deployment convenience).  For callers that cannot allocate device memory:
+ * same arguments and result as sana_linattn_fwd minus the workspace, which is
+ * taken from a fixed array inside the library of
+ * sana_linattn_noalloc_scratch_bytes() bytes (16 MiB) held on every GPU that
+ * loads the library until the process exits.  Shapes needing more scratch
+ * than that (sana_linattn_workspace_size() larger) return
+ * SANA_ERR_UNSUPPORTED.  All calls share the array: calls that overlap on the
+ * GPU (different streams or host threads) race.  The first call on a device
+ * looks up the array's device address; make it before any stream capture.
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_linattn_noalloc_scratch_bytes(void);
+SANA_API sana_status sana_linattn_fwd_noalloc(const sana_shape* shape, sana_dtype dtype,
+                                              const void* q, const void* k, const void* v,
+                                              const void* gate_logits, const sana_rope* rope,
+                                              float eps, void* out, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status helpers.
  * sana_sync_status: synchronizes `stream`, then reports (and clears) the
  * device status word: SANA_ERR_TIMEOUT if a kernel gave up a bounded wait,
