@@ -293,6 +293,16 @@ def components(sana, args):
     ms = time_loop(f, 20)
     out["attnres_route_720p_3src"] = {"ms": ms, "GB_per_s": 4 * TENSOR_BYTES / (ms / 1e3) / 1e9}
     del srcs, h
+    # projection GEMM of the stack: QKVG at 720p, (75,600 x 3072) . (12,288 x 3072)^T
+    A = torch.randn(WL.N, WL.C, device="cuda", dtype=torch.bfloat16)
+    Wq = torch.randn(4 * WL.C, WL.C, device="cuda", dtype=torch.bfloat16) * WL.C ** -0.5
+    Yq = torch.empty(WL.N, 4 * WL.C, device="cuda", dtype=torch.bfloat16)
+    f = lambda: sana.gemm_bf16(A, Wq, out=Yq)
+    for _ in range(3):
+        f()
+    ms = time_loop(f, 10)
+    out["gemm_qkvg_720p"] = {"ms": ms, "TFLOP_per_s": 2 * WL.N * 4 * WL.C * WL.C / (ms / 1e3) / 1e12}
+    del A, Wq, Yq
     # softmax anchor at 720p/5s
     if args.no_anchor:
         out["softmax_anchor_720p"] = {"skipped": "--no-anchor"}
@@ -308,8 +318,33 @@ def components(sana, args):
         ms = time_loop(f, 3)
         flops = 4 * WL.N * WL.N * WL.heads * WL.D
         out["softmax_anchor_720p"] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}
+        del q, k, v, g, y, ws
     except Exception as e:  # not built yet
         out["softmax_anchor_720p"] = {"unavailable": str(e)[:200]}
+    # whole stacks on the 720p/5s grid: the 4-layer 3:1 group (no AttnRes, no
+    # FFN) and the 16-layer AttnRes stack with FFN 3C
+    if args.stacks:
+        grid = (WL.T, WL.H, WL.W)
+        rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
+        for name, layers, attnres, ffn in (("stack_720p_group4", 4, False, 0),
+                                            ("stack_720p_attnres16", 16, True, 3)):
+            x = si.normal(5000 + layers, (1, WL.N, WL.C)).cuda()
+            ws_l = [{k2: t.cuda() for k2, t in d.items()}
+                    for d in si.projection_weights(5, layers, WL.C, ffn)]
+            w_attn, w_ffn = (t.cuda() for t in si.router_queries(5, WL.C))
+            cfg = sana.stack_config(layers, block_span=8, use_attnres=attnres, ffn_mult=ffn)
+            y = torch.empty_like(x)
+            f = lambda: sana.hybrid_stack_fwd(x, ws_l, w_attn, w_ffn, rope, grid, WL.heads, cfg, out=y)
+            f()
+            ms = time_loop(f, 2)
+            nan = 4 * WL.N * WL.N * WL.heads * WL.D
+            lin = 4 * WL.N * WL.heads * WL.D ** 2
+            proj = 2 * WL.N * WL.C * WL.C * (4 + 1 + 2 * ffn)
+            nanc = layers // 4
+            flops = nanc * nan + (layers - nanc) * lin + layers * proj
+            out[name] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12, "layers": layers,
+                         "attnres": attnres, "ffn_mult": ffn}
+            del x, ws_l, y
     return out
 
 
@@ -408,6 +443,22 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_anchor_only(args):
+    """The softmax anchor on the 480p grid (N = 32,760): K steps, ms per call."""
+    import softmax_attention_sana_b200 as sana
+    wl = si.P480
+    q, k, v, g = (t.cuda() for t in si.qkvg(wl))
+    rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
+    y = torch.empty_like(q)
+    f = lambda: sana.softmax_anchor_fwd(q, k, v, g, rope, (wl.T, wl.H, wl.W), wl.heads, out=y)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    flops = 4 * wl.N * wl.N * wl.heads * wl.D
+    print(json.dumps({"anchor_480p_ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,12 +473,19 @@ def main():
                     help="seconds the --impl reference run aims to take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-anchor", action="store_true", help="leave the anchor out of the components")
+    ap.add_argument("--stacks", action="store_true",
+                    help="also time the 4-layer group and the 16-layer AttnRes stack")
+    ap.add_argument("--anchor-only", action="store_true",
+                    help="run only the 480p-shaped softmax anchor (a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup() if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
     try:
+        if args.anchor_only:
+            run_anchor_only(args)
+            return
         if args.impl == "reference":
             run_reference(args, world, rank)
         else:

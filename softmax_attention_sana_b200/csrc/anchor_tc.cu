@@ -5,15 +5,20 @@
 //   Y = sigmoid(G) * softmax(Q' K'^T) V   with Q' = RoPE(Q) * scale * log2(e),
 //   K' = RoPE(K) prepared by a rotation pass, so the softmax works in base 2.
 //
-// One CTA per (batch, head, 128-query tile):
-//   producer warp : TMA Q' and G once, then K' and V tiles (128 keys) in a ring
-//   MMA warp      : S_b = Q' K'_j^T into TMEM buffer b = j % 2 (SS MMA), then
-//                   O += P_{j-1} V_{j-1} with P read from TMEM (TS MMA)
-//   4 softmax warps (thread = query row): online softmax over each S_b row,
-//                   P written back as bf16 into the S_b columns, O rescaled
-//                   in TMEM only when the running max grows by more than
-//                   2^8 (values of P stay <= 256); the epilogue divides by
-//                   the row sum, applies the gate and stores through TMA.
+// One CTA per (batch, head, pair of 128-query tiles).  Both query tiles share
+// every K'/V tile, and their softmax warpgroups ping-pong with the tensor core:
+//   producer warp : TMA Q'_0, Q'_1 once; K'_j, V_j in 2-stage rings; G at the end
+//   MMA warp      : S_0 = Q'_0 K'_0^T, S_1 = Q'_1 K'_0^T, then for each key tile
+//                   j: O_0 += P_0 V_j, S_0 = Q'_0 K'_{j+1}^T, O_1 += P_1 V_j,
+//                   S_1 = Q'_1 K'_{j+1}^T, so one warpgroup's softmax runs while
+//                   the tensor core works for the other
+//   2 x 4 softmax warps (thread = query row of its tile): row max, base-2
+//                   exponentials, P as bf16 written back over its S columns,
+//                   lazy rescaling of O in TMEM (only when a row's max grows
+//                   by more than 2^8, decided warp-uniformly), final 1/l, gate
+//                   and TMA store.
+// TMEM (512 columns): S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512);
+// P_i occupies the first 64 columns of S_i.
 #include <cuda.h>
 
 #include "sana_common.cuh"
@@ -28,7 +33,8 @@ constexpr int kHalf = kRows * 64 * 2;  // 16 KB
 constexpr int kTileB = 2 * kHalf;      // 32 KB
 constexpr int kKS = 2;                 // K' stages
 constexpr int kVS = 2;                 // V stages
-constexpr int kThreads = 192;          // 4 softmax warps + producer + MMA
+constexpr int kThreads = 320;          // 8 softmax warps + producer + MMA
+constexpr int kWarpProd = 8, kWarpMma = 9;
 constexpr float kRescaleLog2 = 8.f;    // lazy rescale threshold (base-2 units)
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -43,12 +49,11 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 struct AnchorCtl {
-  uint64_t q_full;
+  uint64_t q_full, g_full;
   uint64_t k_full[kKS], k_empty[kKS];
   uint64_t v_full[kVS], v_empty[kVS];
-  uint64_t s_full[2], s_free[2], p_full[2];
-  uint64_t pv_done;
-  uint64_t ysync;  // the 128 output rows are staged (bounded wait)
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t ysync[2];  // the 128 output rows of tile i are staged (bounded wait)
   uint32_t tmem;
   int abort_flag;
 };
@@ -61,19 +66,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ AnchorCtl ctl;
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* q_s = smem;                 // Q' tile (later: Y staging when ungated)
-  uint8_t* g_s = q_s + kTileB;         // G tile (Y staging when gated)
-  uint8_t* k_s = g_s + kTileB;         // K' ring
+  uint8_t* q_s = smem;                 // Q'_0, Q'_1 (later: Y staging)
+  uint8_t* k_s = q_s + 2 * kTileB;     // K' ring (later: G tiles)
   uint8_t* v_s = k_s + kKS * kTileB;   // V ring
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int qp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int row0 = qp * 2 * kRows;  // first query row of tile 0
   const int nkv = (N + kRows - 1) / kRows;
   const int kv_tail = N - (nkv - 1) * kRows;  // valid keys in the last tile
   const WaitCtx wc{&ctl.abort_flag, status};
 
   if (tid == 0) {
     mbar_init(&ctl.q_full, 1);
+    mbar_init(&ctl.g_full, 1);
     for (int i = 0; i < kKS; ++i) {
       mbar_init(&ctl.k_full[i], 1);
       mbar_init(&ctl.k_empty[i], 1);
@@ -84,178 +90,221 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.s_full[i], 1);
-      mbar_init(&ctl.s_free[i], 1);
       mbar_init(&ctl.p_full[i], 128);
+      mbar_init(&ctl.pv_done[i], 1);
+      mbar_init(&ctl.ysync[i], 128);
     }
-    mbar_init(&ctl.pv_done, 1);
-    mbar_init(&ctl.ysync, 128);
     ctl.abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(&ctl.tmem, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = ctl.tmem;          // S_0: cols [0,128), S_1: [128,256)
-  const uint32_t tmem_o = tmem + 256;      // O: cols [256, 384)
+  const uint32_t tmem = ctl.tmem;
 
-  if (warp == 4) {
+  if (warp == kWarpProd) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(&ctl.q_full, kGate ? 2 * kTileB : kTileB);
-      tma_load_3d(q_s, &tm_q, &ctl.q_full, h * kD, qt * kRows, b);
-      tma_load_3d(q_s + kHalf, &tm_q, &ctl.q_full, h * kD + 64, qt * kRows, b);
-      if (kGate) {
-        tma_load_3d(g_s, &tm_g, &ctl.q_full, h * kD, qt * kRows, b);
-        tma_load_3d(g_s + kHalf, &tm_g, &ctl.q_full, h * kD + 64, qt * kRows, b);
+      mbar_arrive_expect_tx(&ctl.q_full, 2 * kTileB);
+      for (int i = 0; i < 2; ++i) {
+        tma_load_3d(q_s + i * kTileB, &tm_q, &ctl.q_full, h * kD, row0 + i * kRows, b);
+        tma_load_3d(q_s + i * kTileB + kHalf, &tm_q, &ctl.q_full, h * kD + 64, row0 + i * kRows, b);
       }
-      // K' and V rings advance together; a stage is refilled once the MMAs
-      // that read it have completed.
       int nk = 0, nv = 0;
+      bool ok = true;
       for (int j = 0; j < nkv; ++j) {
         const int sk = j % kKS, sv = j % kVS;
-        if (j >= kKS && !mbar_wait(&ctl.k_empty[sk], ((j / kKS) - 1) & 1, wc, 0x31)) break;
+        if (j >= kKS && !mbar_wait(&ctl.k_empty[sk], ((j / kKS) - 1) & 1, wc, 0x31)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&ctl.k_full[sk], kTileB);
         tma_load_3d(k_s + sk * kTileB, &tm_k, &ctl.k_full[sk], h * kD, j * kRows, b);
         tma_load_3d(k_s + sk * kTileB + kHalf, &tm_k, &ctl.k_full[sk], h * kD + 64, j * kRows, b);
         ++nk;
-        if (j >= kVS && !mbar_wait(&ctl.v_empty[sv], ((j / kVS) - 1) & 1, wc, 0x32)) break;
+        if (j >= kVS && !mbar_wait(&ctl.v_empty[sv], ((j / kVS) - 1) & 1, wc, 0x32)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&ctl.v_full[sv], kTileB);
         tma_load_3d(v_s + sv * kTileB, &tm_v, &ctl.v_full[sv], h * kD, j * kRows, b);
         tma_load_3d(v_s + sv * kTileB + kHalf, &tm_v, &ctl.v_full[sv], h * kD + 64, j * kRows, b);
         ++nv;
       }
+      // G goes into the K ring once the last S MMAs have read it
+      if (ok && kGate) {
+        for (int j = (nkv > kKS ? nkv - kKS : 0); j < nkv && ok; ++j)
+          ok = mbar_wait(&ctl.k_empty[j % kKS], (j / kKS) & 1, wc, 0x3c);
+        if (ok) {
+          mbar_arrive_expect_tx(&ctl.g_full, 2 * kTileB);
+          for (int i = 0; i < 2; ++i) {
+            tma_load_3d(k_s + i * kTileB, &tm_g, &ctl.g_full, h * kD, row0 + i * kRows, b);
+            tma_load_3d(k_s + i * kTileB + kHalf, &tm_g, &ctl.g_full, h * kD + 64,
+                        row0 + i * kRows, b);
+          }
+        }
+      }
       if (*wc.abort_flag) {  // loads still in flight land before the CTA exits
         mbar_drain(&ctl.q_full, 0);
-        for (int j = nk > kKS ? nk - kKS : 0; j < nk; ++j) mbar_drain(&ctl.k_full[j % kKS], (j / kKS) & 1);
-        for (int j = nv > kVS ? nv - kVS : 0; j < nv; ++j) mbar_drain(&ctl.v_full[j % kVS], (j / kVS) & 1);
+        for (int j = nk > kKS ? nk - kKS : 0; j < nk; ++j)
+          mbar_drain(&ctl.k_full[j % kKS], (j / kKS) & 1);
+        for (int j = nv > kVS ? nv - kVS : 0; j < nv; ++j)
+          mbar_drain(&ctl.v_full[j % kVS], (j / kVS) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       // S = Q' K'^T: A = Q' (K-major), B = K' tile (K-major: rows = keys).
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       // O += P V: A = P in TMEM (K-major), B = V tile (MN-major: d contiguous).
       const uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t qb = smem_u32(q_s);
-      bool ok = mbar_wait(&ctl.q_full, 0, wc, 0x33);
-      auto issue_pv = [&](int j) -> bool {  // O += P_j V_j
-        const int bb = j & 1, sv = j % kVS;
-        if (!mbar_wait(&ctl.p_full[bb], (j >> 1) & 1, wc, 0x34)) return false;
-        if (!mbar_wait(&ctl.v_full[sv], (j / kVS) & 1, wc, 0x35)) return false;
-        tc_fence_after();
-        const uint32_t vb = smem_u32(v_s + sv * kTileB);
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          umma_ts(tmem_o, tmem + bb * 128 + kk * 8, smem_desc_sw128(vb + kk * 2048, kHalf, 1024),
-                  idesc_o, (j | kk) != 0);
-        umma_commit(&ctl.pv_done);
-        umma_commit(&ctl.v_empty[sv]);
-        umma_commit(&ctl.s_free[bb]);
-        return true;
-      };
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int bb = j & 1, sk = j % kKS;
-        if (!mbar_wait(&ctl.k_full[sk], (j / kKS) & 1, wc, 0x36)) break;
-        if (j >= 2 && !mbar_wait(&ctl.s_free[bb], ((j >> 1) - 1) & 1, wc, 0x37)) break;
-        tc_fence_after();
-        const uint32_t kb = smem_u32(k_s + sk * kTileB);
+      auto issue_s = [&](int i, int j) {  // S_i = Q'_i K'_j^T
+        const uint32_t qb = smem_u32(q_s + i * kTileB), kb = smem_u32(k_s + (j % kKS) * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_ss(tmem + bb * 128, smem_desc_sw128(qb + off, 16, 1024),
+          umma_ss(tmem + i * 128, smem_desc_sw128(qb + off, 16, 1024),
                   smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk != 0);
         }
-        umma_commit(&ctl.s_full[bb]);
-        umma_commit(&ctl.k_empty[sk]);
-        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+        umma_commit(&ctl.s_full[i]);
+      };
+      auto issue_pv = [&](int i, int j) {  // O_i += P_i V_j
+        const uint32_t vb = smem_u32(v_s + (j % kVS) * kTileB);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          umma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
+                  smem_desc_sw128(vb + kk * 2048, kHalf, 1024), idesc_o, (j | kk) != 0);
+        umma_commit(&ctl.pv_done[i]);
+      };
+      bool ok = mbar_wait(&ctl.q_full, 0, wc, 0x33) && nkv > 0 &&
+                mbar_wait(&ctl.k_full[0], 0, wc, 0x36);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(&ctl.k_empty[0]);  // K'_0 is read by these two only
       }
-      if (ok && nkv > 0) issue_pv(nkv - 1);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const bool more = j + 1 < nkv;
+        if (!mbar_wait(&ctl.v_full[j % kVS], (j / kVS) & 1, wc, 0x35)) break;
+        if (more && !mbar_wait(&ctl.k_full[(j + 1) % kKS], ((j + 1) / kKS) & 1, wc, 0x36)) break;
+        for (int i = 0; i < 2 && ok; ++i) {
+          // P_i of tile j is in TMEM; O_i has been rescaled if needed
+          if (!mbar_wait(&ctl.p_full[i], j & 1, wc, 0x34)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(i, j);
+          if (more) {
+            // S_i is overwritten only after the MMAs that read P_i from it finish
+            if (!mbar_wait(&ctl.pv_done[i], j & 1, wc, 0x37)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(i, j + 1);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&ctl.v_empty[j % kVS]);
+        if (more) umma_commit(&ctl.k_empty[(j + 1) % kKS]);
+      }
     }
   } else {
     // ------------------------------------------------ softmax warps: thread = query row
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int qi = warp >> 2;                 // which query tile
+    const int r = (warp & 3) * 32 + lane;     // row within the tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tmem_s = tmem + qi * 128, tmem_o = tmem + 256 + qi * 128;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; ok && j < nkv; ++j) {
-      const int bb = j & 1;
       // warp-uniform outcome: tcgen05.ld / st are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&ctl.s_full[bb], (j >> 1) & 1, wc, 0x38))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl.s_full[qi], j & 1, wc, 0x38))) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + bb * 128 + c * 32, sr[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
       tmem_ld_wait();
-      const int valid = (j == nkv - 1) ? kv_tail : kRows;
       float mx = -INFINITY;
+      if (j == nkv - 1 && kv_tail < kRows) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float s = __uint_as_float(sr[c][i]);
-          if (c * 32 + i >= valid) s = -INFINITY;
-          sr[c][i] = __float_as_uint(s);
-          mx = fmaxf(mx, s);
-        }
-      const float m_new = fmaxf(m, mx);
-      // rescale O when any row of the warp needs it (collective TMEM access)
-      const bool grow = m_new > m + kRescaleLog2;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float m_use = grow ? m_new : m;
-        const float corr = ex2(m - m_use);  // 0 on the first tile, 1 for rows that keep m
-        if (j >= 1) {
-          // O holds the sum over tiles < j; wait for the last PV before touching it
-          if (!__all_sync(0xffffffffu, mbar_wait(&ctl.pv_done, (j - 1) & 1, wc, 0x39))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem_o + lane_base + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-            tmem_st32(tmem_o + lane_base + c * 32, o);
-          }
-          tmem_st_wait();
-        }
-        l *= corr;
-        m = m_use;
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= kv_tail) sr[c][i] = __float_as_uint(-INFINITY);
       }
-      float rs = 0.f;
-      uint32_t pk[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+      const float m_new = fmaxf(m, mx);
+      // lazy rescaling: a row moves its reference max only when the max grew
+      // by more than 2^8; the decision to touch O is warp-uniform because TMEM
+      // access is warp-collective (rows that keep their max use a factor 1)
+      const bool grow = m_new > m + kRescaleLog2;
+      const bool any_grow = __any_sync(0xffffffffu, grow);
+      const float m_use = grow ? m_new : m;
+      const float corr = ex2(m - m_use);  // 0 on the first tile
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2(__uint_as_float(sr[c][i]) - m);
-          const float p1 = ex2(__uint_as_float(sr[c][i + 1]) - m);
+          const float p0 = ex2(__uint_as_float(sr[c][i]) - m_use);
+          const float p1 = ex2(__uint_as_float(sr[c][i + 1]) - m_use);
           rs += p0 + p1;
-          pk[c >> 1][(c & 1) * 16 + i / 2] = f2_to_bf2(p0, p1);
+          pk[i / 2] = f2_to_bf2(p0, p1);
         }
-      l += rs;
-      tmem_st32(tmem + lane_base + bb * 128, pk[0]);
-      tmem_st32(tmem + lane_base + bb * 128 + 32, pk[1]);
+        // P columns: key k lives in column k / 2 of S_i
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sr[c >> 1][(c & 1) * 16 + i] = pk[i];
+      }
+      l = l * corr + rs;
+      m = m_use;
+      tmem_st32(tmem_s + lane_base, sr[0]);
+      tmem_st32(tmem_s + lane_base + 32, sr[1]);
+      if (any_grow && j >= 1) {
+        // O_i holds the sum over tiles < j (their PV MMAs finished before S_i
+        // of this tile was issued); scale it before the next PV accumulates
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctl.pv_done[qi], (j - 1) & 1, wc, 0x39))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_base + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+          tmem_st32(tmem_o + lane_base + c * 32, o);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ctl.p_full[bb]);
+      mbar_arrive(&ctl.p_full[qi]);
     }
     // ---------------- epilogue: Y = O / l * sigmoid(G)
-    ok = __all_sync(0xffffffffu, ok && nkv > 0 && mbar_wait(&ctl.pv_done, (nkv - 1) & 1, wc, 0x3a));
-    uint8_t* ybuf = kGate ? g_s : q_s;
+    ok = __all_sync(0xffffffffu,
+                    ok && nkv > 0 && mbar_wait(&ctl.pv_done[qi], (nkv - 1) & 1, wc, 0x3a));
+    if (kGate) ok = ok && __all_sync(0xffffffffu, mbar_wait(&ctl.g_full, 0, wc, 0x3d));
+    uint8_t* ybuf = q_s + qi * kTileB;  // Q'_i is no longer read
+    const uint8_t* gbuf = k_s + qi * kTileB;
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l;
@@ -264,14 +313,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[32];
         tmem_ld32(tmem_o + lane_base + c * 32, o);
         tmem_ld_wait();
-        uint8_t* hb = ybuf + (c >> 1) * kHalf;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // 8 columns per 16-byte chunk
           const int ch = (c & 1) * 4 + q;
-          uint4* p = reinterpret_cast<uint4*>(hb + sw128_off(r, ch));
+          const uint32_t off = (c >> 1) * kHalf + sw128_off(r, ch);
           uint32_t gw[4] = {0, 0, 0, 0};
           if (kGate) {
-            const uint4 gr = *p;
+            const uint4 gr = *reinterpret_cast<const uint4*>(gbuf + off);
             gw[0] = gr.x; gw[1] = gr.y; gw[2] = gr.z; gw[3] = gr.w;
           }
           uint32_t out[4];
@@ -286,24 +334,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             out[i] = f2_to_bf2(y0, y1);
           }
-          *p = make_uint4(out[0], out[1], out[2], out[3]);
+          *reinterpret_cast<uint4*>(ybuf + off) = make_uint4(out[0], out[1], out[2], out[3]);
         }
       }
       fence_proxy_async_smem();
     }
-    mbar_arrive(&ctl.ysync);
-    ok = mbar_wait(&ctl.ysync, 0, wc, 0x3b) && ok;
-    if (ok && tid == 0) {
-      tma_store_3d(&tm_y, ybuf, h * kD, qt * kRows, b);
-      tma_store_3d(&tm_y, ybuf + kHalf, h * kD + 64, qt * kRows, b);
+    mbar_arrive(&ctl.ysync[qi]);
+    ok = mbar_wait(&ctl.ysync[qi], 0, wc, 0x3b) && ok;
+    if (ok && r == 0 && row0 + qi * kRows < N) {  // a tile past N has nothing to store
+      tma_store_3d(&tm_y, ybuf, h * kD, row0 + qi * kRows, b);
+      tma_store_3d(&tm_y, ybuf + kHalf, h * kD + 64, row0 + qi * kRows, b);
       bulk_commit();
       bulk_wait0();
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
-    if (*wc.abort_flag) mbar_drain(&ctl.pv_done, (nkv - 1) & 1);
+  if (warp == kWarpMma) {
+    if (*wc.abort_flag) {  // MMAs in flight finish before TMEM is freed
+      mbar_drain(&ctl.pv_done[0], (nkv - 1) & 1);
+      mbar_drain(&ctl.pv_done[1], (nkv - 1) & 1);
+    }
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -334,7 +385,8 @@ sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr,
                          (int)kAnchorSmem);
     attr[dev] = true;
   }
-  const dim3 grid((g.N + kRows - 1) / kRows, s.heads, s.B);
+  const int qtiles = (g.N + kRows - 1) / kRows;
+  const dim3 grid((qtiles + 1) / 2, s.heads, s.B);
   if (gt)
     anchor_kernel<true><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, status_word());
   else

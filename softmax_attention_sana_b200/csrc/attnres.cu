@@ -159,6 +159,121 @@ __global__ void __launch_bounds__(MAXS <= 4 ? 1024 : 512)
   }
 }
 
+// Warp per token, the token's row of every source held in registers (bf16,
+// NS <= 4 sources, C <= 256 * CH): one HBM read of each source, warp-shuffle
+// reductions only, several tokens in flight per SM.
+template <int NS, int CH>
+__global__ void __launch_bounds__(256)
+    attnres_warp_kernel(SourcePtrs src, long long tokens, int C, const float* __restrict__ w,
+                        float eps, __nv_bfloat16* __restrict__ h_out, float* __restrict__ alpha_out,
+                        __nv_bfloat16* __restrict__ hn_out) {
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  const float invC = 1.f / (float)C;
+  for (long long tok = warp0; tok < tokens; tok += nwarps) {
+    const size_t row = (size_t)tok * C;
+    uint4 x[NS][CH];
+#pragma unroll
+    for (int s = 0; s < NS; ++s)
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = (c * 32 + lane) * 8;
+        x[s][c] = col < C ? *reinterpret_cast<const uint4*>(
+                                static_cast<const __nv_bfloat16*>(src.p[s]) + row + col)
+                          : make_uint4(0, 0, 0, 0);
+      }
+    float ss[NS], sw[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) ss[s] = sw[s] = 0.f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * 32 + lane) * 8;
+      if (col >= C) continue;
+      const float4 w0 = *reinterpret_cast<const float4*>(w + col);
+      const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
+      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf2_to_f2(u[i]);
+          ss[s] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss[s]));
+          sw[s] = fmaf(wv[2 * i], f.x, fmaf(wv[2 * i + 1], f.y, sw[s]));
+        }
+      }
+    }
+    float a[NS], m = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss[s] += __shfl_xor_sync(0xffffffffu, ss[s], o);
+        sw[s] += __shfl_xor_sync(0xffffffffu, sw[s], o);
+      }
+      a[s] = sw[s] * rsqrtf(ss[s] * invC + eps);
+      m = fmaxf(m, a[s]);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      a[s] = expf(a[s] - m);
+      den += a[s];
+    }
+    const float inv = 1.f / den;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      a[s] *= inv;
+      if (alpha_out && lane == s) alpha_out[(size_t)tok * NS + s] = a[s];
+    }
+    // h = sum_s a_s v_s, chunk by chunk from the registers
+    float hss = 0.f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * 32 + lane) * 8;
+      float hv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf2_to_f2(u[i]);
+          hv[2 * i] = fmaf(a[s], f.x, hv[2 * i]);
+          hv[2 * i + 1] = fmaf(a[s], f.y, hv[2 * i + 1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hss = fmaf(hv[i], hv[i], hss);
+      if (h_out && col < C) Vec8<__nv_bfloat16>::store(h_out + row + col, hv);
+    }
+    if (hn_out) {  // fused pre-norm of the routed representation (h recomputed)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) hss += __shfl_xor_sync(0xffffffffu, hss, o);
+      const float rn = rsqrtf(hss * invC + eps);
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = (c * 32 + lane) * 8;
+        if (col >= C) continue;
+        float hv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = bf2_to_f2(u[i]);
+            hv[2 * i] = fmaf(a[s], f.x, hv[2 * i]);
+            hv[2 * i + 1] = fmaf(a[s], f.y, hv[2 * i + 1]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hv[i] *= rn;
+        Vec8<__nv_bfloat16>::store(hn_out + row + col, hv);
+      }
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(1024)
     rmsnorm_kernel(const T* __restrict__ x, long long rows, int C, float eps, T* __restrict__ y) {
@@ -190,9 +305,45 @@ int threads_for(int C) {
   return t < 32 ? 32 : t;
 }
 
+template <int NS, int CH>
+void warp_launch(const SourcePtrs& sp, long long tokens, int C, const float* w, float eps, void* h,
+                 float* alpha, void* hn, cudaStream_t st) {
+  const long long warps = tokens < (long long)kNumSMs * 64 ? tokens : (long long)kNumSMs * 64;
+  attnres_warp_kernel<NS, CH><<<(int)((warps + 7) / 8), 256, 0, st>>>(
+      sp, tokens, C, w, eps, static_cast<__nv_bfloat16*>(h), alpha,
+      static_cast<__nv_bfloat16*>(hn));
+}
+
+template <int CH>
+bool warp_launch_s(const SourcePtrs& sp, int S, long long tokens, int C, const float* w, float eps,
+                   void* h, float* alpha, void* hn, cudaStream_t st) {
+  switch (S) {
+    case 1: warp_launch<1, CH>(sp, tokens, C, w, eps, h, alpha, hn, st); return true;
+    case 2: warp_launch<2, CH>(sp, tokens, C, w, eps, h, alpha, hn, st); return true;
+    case 3: warp_launch<3, CH>(sp, tokens, C, w, eps, h, alpha, hn, st); return true;
+    case 4: warp_launch<4, CH>(sp, tokens, C, w, eps, h, alpha, hn, st); return true;
+  }
+  return false;
+}
+
+// bf16, <= 4 sources, C a multiple of 256 up to 4096: warp per token.
+bool launch_attnres_warp(const SourcePtrs& sp, int S, long long tokens, int C, const float* w,
+                         float eps, void* h, float* alpha, void* hn, cudaStream_t st) {
+  const int ch = C / 256;
+  if (ch <= 4) return warp_launch_s<4>(sp, S, tokens, C, w, eps, h, alpha, hn, st);
+  if (ch <= 8) return warp_launch_s<8>(sp, S, tokens, C, w, eps, h, alpha, hn, st);
+  if (ch <= 12) return warp_launch_s<12>(sp, S, tokens, C, w, eps, h, alpha, hn, st);
+  return warp_launch_s<16>(sp, S, tokens, C, w, eps, h, alpha, hn, st);
+}
+
 template <typename T>
 void launch_attnres(const SourcePtrs& sp, int S, long long tokens, int C, const float* w, float eps,
                     void* h, float* alpha, void* hn, cudaStream_t st) {
+  if constexpr (sizeof(T) == 2) {
+    if (S <= 4 && C <= 4096 && C % 256 == 0 && launch_attnres_warp(sp, S, tokens, C, w, eps, h,
+                                                                    alpha, hn, st))
+      return;
+  }
   const int threads = threads_for(C);
   long long blocks = tokens < (long long)kNumSMs * 16 ? tokens : (long long)kNumSMs * 16;
   if (blocks < 1) blocks = 1;

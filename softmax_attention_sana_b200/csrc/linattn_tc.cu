@@ -11,14 +11,22 @@
 //           ReLU + RoPE of K in shared memory (z accumulated on the way) ->
 //           tcgen05 D[d][e] += K'^T V with fp32 accumulation in TMEM ->
 //           partial S and z to the workspace.
-//   combine per (batch, head): fixed-order sum of the split partials (plus the
-//           carried state in block-causal mode) into S and z in fp32.
+//   combine per (batch, head, slice of S): fixed-order sum of the split
+//           partials (plus the carried state in block-causal mode).
 //   output  per (batch, head, split): S (fp32) -> bf16 S^T operand in shared
 //           memory once per CTA; TMA Q, G tiles -> ReLU + RoPE of Q and the
 //           RoPE-free denominator phi(Q).z in registers -> tcgen05 D = Q' S ->
 //           epilogue divides, gates with sigmoid(G), stores bf16 through
 //           shared memory with TMA.
+//
+// Workers are 16 warps: warp w owns TMEM lane quarter w % 4 (token rows
+// 32(w%4) .. +31) and column quarter w / 4 (32 of the 128 head dims), so each
+// thread transforms one 64-byte run of one token row per tile.  The rotary
+// split 22/21/21 of the 128-dim heads is compiled in (pair-to-axis selection
+// folds away); other splits take the general path.
 #include <cuda.h>
+
+#include <cstddef>
 
 #include "rope_dev.cuh"
 #include "sana_common.cuh"
@@ -31,20 +39,31 @@ constexpr int kD = 128;
 constexpr int kRows = 128;                // tokens per tile
 constexpr int kHalf = kRows * 64 * 2;     // one 64-column half of a tile: 16 KB
 constexpr int kTileB = 2 * kHalf;         // 32 KB
-constexpr int kWorkers = 256;             // 8 warps: (row quarter, column half)
+constexpr int kWorkers = 512;             // 16 warps: (row quarter, column quarter)
 constexpr int kThreadsA = kWorkers + 64;  // + producer warp + MMA warp
 constexpr int kStagesA = 3;
 constexpr int kStagesQ = 3;
 constexpr int kStagesG = 2;
 constexpr int kThreadsB = kWorkers + 96;  // + Q producer, MMA, G producer
+constexpr int kWarpProdA = 16, kWarpMmaA = 17;
+constexpr int kWarpProdQ = 16, kWarpMmaB = 17, kWarpProdG = 18;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// ReLU + RoPE of one 16-byte chunk (4 rotary pairs) of a swizzled tile row,
-// rewritten in place.  phi values are returned for z / the denominator.
+// (cos, sin) of rotary pair j.  NT >= 0: the split is a compile-time constant
+// and, with j unrolled, the axis selection is resolved by the compiler.
+template <int NT, int NH>
+__device__ __forceinline__ float2 pair_cs(const RowRope& rr, int j) {
+  if (NT >= 0) return j < NT ? rr.pt[j] : (j < NT + NH ? rr.ph[j - NT] : rr.pw[j - NT - NH]);
+  return rr.cs(j);
+}
+
+// ReLU + RoPE of one 16-byte chunk (4 rotary pairs starting at pair0) of a
+// swizzled tile row, rewritten in place; the ReLU values are returned.
+template <int NT, int NH>
 __device__ __forceinline__ void relu_rope_chunk(uint8_t* p, const RowRope& rr, int pair0,
                                                 float (&phi_out)[8]) {
   uint4 raw = *reinterpret_cast<uint4*>(p);
@@ -56,10 +75,47 @@ __device__ __forceinline__ void relu_rope_chunk(uint8_t* p, const RowRope& rr, i
     x.y = fmaxf(x.y, 0.f);
     phi_out[2 * i] = x.x;
     phi_out[2 * i + 1] = x.y;
-    const float2 r = rotate(x.x, x.y, rr.cs(pair0 + i));
+    const float2 r = rotate(x.x, x.y, pair_cs<NT, NH>(rr, pair0 + i));
     w[i] = f2_to_bf2(r.x, r.y);
   }
   *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Column quarter C4 of token row r: chunks 4*(C4&1) .. +3 of half C4>>1.
+template <int NT, int NH, int C4>
+__device__ __forceinline__ void quarter_state(uint8_t* tile, int r, const RowRope& rr,
+                                              float (&zacc)[32]) {
+  uint8_t* half = tile + (C4 >> 1) * kHalf;
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    float ph[8];
+    relu_rope_chunk<NT, NH>(half + sw128_off(r, (C4 & 1) * 4 + ch), rr, C4 * 16 + ch * 4, ph);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) zacc[ch * 8 + i] += ph[i];
+  }
+}
+
+template <int NT, int NH, int C4>
+__device__ __forceinline__ float quarter_query(uint8_t* tile, int r, const RowRope& rr,
+                                               const float* z) {
+  uint8_t* half = tile + (C4 >> 1) * kHalf;
+  float den = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    float ph[8];
+    relu_rope_chunk<NT, NH>(half + sw128_off(r, (C4 & 1) * 4 + ch), rr, C4 * 16 + ch * 4, ph);
+    const float4 z0 = *reinterpret_cast<const float4*>(z + C4 * 32 + ch * 8);
+    const float4 z1 = *reinterpret_cast<const float4*>(z + C4 * 32 + ch * 8 + 4);
+    den = fmaf(ph[0], z0.x, den);
+    den = fmaf(ph[1], z0.y, den);
+    den = fmaf(ph[2], z0.z, den);
+    den = fmaf(ph[3], z0.w, den);
+    den = fmaf(ph[4], z1.x, den);
+    den = fmaf(ph[5], z1.y, den);
+    den = fmaf(ph[6], z1.z, den);
+    den = fmaf(ph[7], z1.w, den);
+  }
+  return den;
 }
 
 // ------------------------------------------------------------------------
@@ -74,6 +130,7 @@ struct StateSmemCtl {
   int abort_flag;
 };
 
+template <int NT, int NH>
 __global__ void __launch_bounds__(kThreadsA, 1)
     linattn_state_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, RopeDev rope, GridDev g,
@@ -102,7 +159,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     ctl.abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 9) {
+  if (warp == kWarpMmaA) {
     tmem_alloc(&ctl.tmem, 128);
     tmem_relinquish();
   }
@@ -112,7 +169,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   tc_fence_after();
   const uint32_t tmem = ctl.tmem;
 
-  if (warp == 8) {
+  if (warp == kWarpProdA) {
     // ---------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_k);
@@ -132,12 +189,11 @@ __global__ void __launch_bounds__(kThreadsA, 1)
         ++issued;
       }
       if (*abort_flag) {  // drain loads still in flight before the CTA exits
-        for (int it = issued > kStagesA ? issued - kStagesA : 0; it < issued; ++it) {
+        for (int it = issued > kStagesA ? issued - kStagesA : 0; it < issued; ++it)
           mbar_drain(&ctl.full[it % kStagesA], (it / kStagesA) & 1);
-        }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kWarpMmaA) {
     // ---------------- MMA issuer: D[d][e] += K'[tok][d]^T V[tok][e]
     if (lane == 0) {
       // A = K' (M = d, MN-major), B = V (N = e, MN-major), both 128B-swizzled
@@ -160,25 +216,24 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       }
       umma_commit(&ctl.done);
     }
-  } else {
-    // ---------------- workers: thread = (token row r, column half c)
-    const int q4 = warp & 3, c = warp >> 2, r = q4 * 32 + lane;
-    float zacc[64];
+  } else if (warp < 16) {
+    // ---------------- workers: thread = (token row r, column quarter c4)
+    const int q4 = warp & 3, c4 = warp >> 2, r = q4 * 32 + lane;
+    float zacc[32];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) zacc[i] = 0.f;
+    for (int i = 0; i < 32; ++i) zacc[i] = 0.f;
     for (int it = 0; it < ntiles; ++it) {
       const int s = it % kStagesA;
       if (!mbar_wait(&ctl.full[s], (it / kStagesA) & 1, wc, 0x13)) break;
       const int n = (tile0 + it) * kRows + r;
       if (n < g.N) {  // rows past N were zero-filled by TMA: phi = RoPE = 0
         const RowRope rr = row_rope(rs, g, n);
-        uint8_t* half = stages + s * 2 * kTileB + c * kHalf;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          float ph[8];
-          relu_rope_chunk(half + sw128_off(r, ch), rr, c * 32 + ch * 4, ph);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) zacc[ch * 8 + i] += ph[i];
+        uint8_t* tile = stages + s * 2 * kTileB;
+        switch (c4) {  // warp-uniform
+          case 0: quarter_state<NT, NH, 0>(tile, r, rr, zacc); break;
+          case 1: quarter_state<NT, NH, 1>(tile, r, rr, zacc); break;
+          case 2: quarter_state<NT, NH, 2>(tile, r, rr, zacc); break;
+          default: quarter_state<NT, NH, 3>(tile, r, rr, zacc); break;
         }
       }
       fence_proxy_async_smem();
@@ -189,34 +244,31 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     const size_t part = ((size_t)(b * g.heads + h) * splits + split);
     if (ok) {
       float* Sout = ws_S + part * kD * kD;
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c4 * 32, v);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(Sout + (size_t)r * kD + c4 * 32);
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c * 64 + j * 32, v);
-        tmem_ld_wait();
-        float4* dst = reinterpret_cast<float4*>(Sout + (size_t)r * kD + c * 64 + j * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-      }
+      for (int i = 0; i < 8; ++i)
+        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
     }
-    // z: reduce the per-row partial sums over the 128 rows of each half in a
-    // fixed order (stride 65 keeps both passes free of bank conflicts).
+    // z: reduce the per-row partial sums over the 128 rows of each column
+    // quarter in a fixed order (stride 33 keeps both passes conflict-free).
     float* red = reinterpret_cast<float*>(stages);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) red[(c * 128 + r) * 65 + i] = zacc[i];
+    for (int i = 0; i < 32; ++i) red[(c4 * 128 + r) * 33 + i] = zacc[i];
     named_bar_sync(1, kWorkers);
     if (tid < 128) {
-      const int cc = tid >> 6, i = tid & 63;
+      const int cc = tid >> 5, i = tid & 31;
       float acc = 0.f;
-      for (int rr = 0; rr < 128; ++rr) acc += red[(cc * 128 + rr) * 65 + i];
-      ws_z[part * kD + cc * 64 + i] = acc;
+      for (int rr = 0; rr < 128; ++rr) acc += red[(cc * 128 + rr) * 33 + i];
+      ws_z[part * kD + cc * 32 + i] = acc;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMmaA) {
     if (*abort_flag) mbar_drain(&ctl.done, 0);  // MMAs in flight finish before TMEM is freed
     tc_fence_after();
     tmem_dealloc(tmem, 128);
@@ -224,27 +276,35 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 }
 
 // ------------------------------------------------------------------------
-// combine kernel (shared with the fp32 path): fixed-order sum over splits
+// combine kernel (shared with the fp32 path): fixed-order sum over splits.
+// Grid (batch * heads, slices): each CTA sums one slice of one head's S.
 // ------------------------------------------------------------------------
-__global__ void linattn_combine_kernel(const float* __restrict__ ws_S,
-                                       const float* __restrict__ ws_z, int splits, int D,
-                                       const float* S_prev, const float* z_prev, float* S_state,
-                                       float* z_state, float* __restrict__ S_f32,
-                                       float* __restrict__ z_out) {
+constexpr int kCombineSlices = 16;
+
+__global__ void __launch_bounds__(256)
+    linattn_combine_kernel(const float* __restrict__ ws_S, const float* __restrict__ ws_z,
+                           int splits, int D, const float* S_prev, const float* z_prev,
+                           float* S_state, float* z_state, float* __restrict__ S_f32,
+                           float* __restrict__ z_out) {
   const int bh = blockIdx.x;
-  const size_t DD = (size_t)D * D;
-  for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x) {
-    float acc = S_prev ? S_prev[bh * DD + idx] : 0.f;
+  const int DD = D * D;
+  const int per = (DD + (int)gridDim.y - 1) / (int)gridDim.y;
+  const int beg = (int)blockIdx.y * per;
+  const int end = min(DD, beg + per);
+  const size_t base = (size_t)bh * DD;
+  for (int idx = beg + threadIdx.x; idx < end; idx += blockDim.x) {
+    float acc = S_prev ? S_prev[base + idx] : 0.f;
     for (int sp = 0; sp < splits; ++sp) acc += ws_S[((size_t)bh * splits + sp) * DD + idx];
-    if (S_state) S_state[bh * DD + idx] = acc;
-    if (S_f32) S_f32[bh * DD + idx] = acc;
+    if (S_state) S_state[base + idx] = acc;
+    if (S_f32) S_f32[base + idx] = acc;
   }
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = z_prev ? z_prev[(size_t)bh * D + d] : 0.f;
-    for (int sp = 0; sp < splits; ++sp) acc += ws_z[((size_t)bh * splits + sp) * D + d];
-    if (z_state) z_state[(size_t)bh * D + d] = acc;
-    if (z_out) z_out[(size_t)bh * D + d] = acc;
-  }
+  if (blockIdx.y == 0)
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float acc = z_prev ? z_prev[(size_t)bh * D + d] : 0.f;
+      for (int sp = 0; sp < splits; ++sp) acc += ws_z[((size_t)bh * splits + sp) * D + d];
+      if (z_state) z_state[(size_t)bh * D + d] = acc;
+      if (z_out) z_out[(size_t)bh * D + d] = acc;
+    }
 }
 
 // ------------------------------------------------------------------------
@@ -257,11 +317,12 @@ struct OutSmemCtl {
   uint64_t wsync, hsync[2];  // reusable worker barriers (bounded waits)
   uint32_t tmem;
   int abort_flag;
-  float den[kStagesQ][2][kRows];
-  float z[kD];
+  alignas(16) float den[kStagesQ][4][kRows];
+  alignas(16) float z[kD];  // read as float4
 };
+static_assert(offsetof(OutSmemCtl, z) % 16 == 0, "z is read with 16-byte loads");
 
-template <bool kGate>
+template <bool kGate, int NT, int NH>
 __global__ void __launch_bounds__(kThreadsB, 1)
     linattn_out_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_g,
@@ -296,30 +357,31 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.mma_done[i], 1);
       mbar_init(&ctl.tmem_free[i], kWorkers);
-      mbar_init(&ctl.hsync[i], 128);
+      mbar_init(&ctl.hsync[i], kWorkers / 2);
     }
     mbar_init(&ctl.wsync, kWorkers);
     ctl.abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 9) {
+  if (warp == kWarpMmaB) {
     tmem_alloc(&ctl.tmem, 256);
     tmem_relinquish();
   }
   if (tid < kD) ctl.z[tid] = z_all[(size_t)bh * kD + tid];
   if (tid < kWorkers) {
     // S^T operand: element (e, d) = S[d][e] in bf16, K-major [2 halves of
-    // 64 d][128 e rows] with the 128-byte swizzle.  Thread = (row e, half).
-    const int e = tid & 127, hf = tid >> 7;
-    const float* Sh = S_all + (size_t)bh * kD * kD + (size_t)(hf * 64) * kD + e;
-    uint8_t* dst = s_op + hf * kHalf;
-#pragma unroll 2
-    for (int ch = 0; ch < 8; ++ch) {
+    // 64 d][128 e rows] with the 128-byte swizzle.  Thread = (row e, d quarter).
+    const int e = tid & 127, qd = tid >> 7;
+    const float* Sh = S_all + (size_t)bh * kD * kD + (size_t)(qd * 32) * kD + e;
+    uint8_t* dst = s_op + (qd >> 1) * kHalf;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
       uint32_t wv[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         wv[i] = f2_to_bf2(Sh[(ch * 8 + 2 * i) * kD], Sh[(ch * 8 + 2 * i + 1) * kD]);
-      *reinterpret_cast<uint4*>(dst + sw128_off(e, ch)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      *reinterpret_cast<uint4*>(dst + sw128_off(e, (qd & 1) * 4 + ch)) =
+          make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
     fence_proxy_async_smem();
   }
@@ -329,7 +391,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   tc_fence_after();
   const uint32_t tmem = ctl.tmem;
 
-  if (warp == 8) {
+  if (warp == kWarpProdQ) {
     // ---------------- Q producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -343,7 +405,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tma_load_3d(q_st + s * kTileB + kHalf, &tm_q, &ctl.fullQ[s], h * kD + 64, n0, b);
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == kWarpProdG) {
     // ---------------- G producer (ungated: only hands out the staging buffers)
     if (lane == 0) {
       if (kGate) prefetch_tmap(&tm_g);
@@ -361,7 +423,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kWarpMmaB) {
     // ---------------- MMA issuer: D[tok][e] = Q'[tok][d] S[d][e]
     if (lane == 0) {
       // A = Q' (K-major, [2 halves][128 tok][64 d]), B = S^T (K-major,
@@ -384,9 +446,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         umma_commit(&ctl.mma_done[tb]);
       }
     }
-  } else {
-    // ---------------- workers: thread = (token row r, column half c)
-    const int q4 = warp & 3, c = warp >> 2, r = q4 * 32 + lane;
+  } else if (warp < 16) {
+    // ---------------- workers: thread = (token row r, column quarter c4)
+    const int q4 = warp & 3, c4 = warp >> 2, r = q4 * 32 + lane;
+    const int hf = c4 >> 1;  // the 64-column half holding this thread's columns
     bool ok = true;
     auto prologue = [&](int it) {
       const int s = it % kStagesQ;
@@ -398,16 +461,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       float den = 0.f;
       if (n < g.N) {
         const RowRope rr = row_rope(rs, g, n);
-        uint8_t* half = q_st + s * kTileB + c * kHalf;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          float ph[8];
-          relu_rope_chunk(half + sw128_off(r, ch), rr, c * 32 + ch * 4, ph);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) den = fmaf(ph[i], ctl.z[c * 64 + ch * 8 + i], den);
+        uint8_t* tile = q_st + s * kTileB;
+        switch (c4) {  // warp-uniform
+          case 0: den = quarter_query<NT, NH, 0>(tile, r, rr, ctl.z); break;
+          case 1: den = quarter_query<NT, NH, 1>(tile, r, rr, ctl.z); break;
+          case 2: den = quarter_query<NT, NH, 2>(tile, r, rr, ctl.z); break;
+          default: den = quarter_query<NT, NH, 3>(tile, r, rr, ctl.z); break;
         }
       }
-      ctl.den[s][c][r] = den;
+      ctl.den[s][c4][r] = den;
       fence_proxy_async_smem();
       mbar_arrive(&ctl.qready[s]);
     };
@@ -415,26 +477,26 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     auto epilogue = [&](int it) {
       const int s = it % kStagesQ, tb = it & 1, sg = it % kStagesG;
       bool okw = mbar_wait(&ctl.mma_done[tb], (it >> 1) & 1, wc, 0x27);
-      // both column halves have written their partial denominators
+      // every column quarter has written its partial denominator
       mbar_arrive(&ctl.wsync);
       okw = mbar_wait(&ctl.wsync, (n_wsync++) & 1, wc, 0x29) && okw;
       okw = __all_sync(0xffffffffu, okw);  // tcgen05.ld is warp-collective
-      const float inv = 1.f / (ctl.den[s][0][r] + ctl.den[s][1][r] + eps);
-      uint32_t acc[2][32];
+      const float inv =
+          1.f / (ctl.den[s][0][r] + ctl.den[s][1][r] + ctl.den[s][2][r] + ctl.den[s][3][r] + eps);
+      uint32_t acc[32];
       if (okw) {
         tc_fence_after();
-        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 128 + c * 64, acc[0]);
-        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 128 + c * 64 + 32, acc[1]);
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + tb * 128 + c4 * 32, acc);
         tmem_ld_wait();
       }
       tc_fence_before();
       mbar_arrive(&ctl.tmem_free[tb]);
       okw = mbar_wait(&ctl.fullG[sg], (it / kStagesG) & 1, wc, 0x28) && okw;
-      uint8_t* half = g_st + sg * kTileB + c * kHalf;
+      uint8_t* half = g_st + sg * kTileB + hf * kHalf;
       if (okw) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4* p = reinterpret_cast<uint4*>(half + sw128_off(r, ch));
+        for (int ch = 0; ch < 4; ++ch) {
+          uint4* p = reinterpret_cast<uint4*>(half + sw128_off(r, (c4 & 1) * 4 + ch));
           uint32_t gw[4] = {0, 0, 0, 0};
           if (kGate) {
             const uint4 graw = *p;
@@ -443,9 +505,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           uint32_t out[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int col = (ch & 3) * 8 + 2 * i;
-            float y0 = __uint_as_float(acc[ch >> 2][col]) * inv;
-            float y1 = __uint_as_float(acc[ch >> 2][col + 1]) * inv;
+            float y0 = __uint_as_float(acc[ch * 8 + 2 * i]) * inv;
+            float y1 = __uint_as_float(acc[ch * 8 + 2 * i + 1]) * inv;
             if (kGate) {
               const float2 gg = bf2_to_f2(gw[i]);
               y0 *= sigmoid_fast(gg.x);
@@ -457,11 +518,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
       }
       fence_proxy_async_smem();
-      // the 128 rows of this column half are staged
-      mbar_arrive(&ctl.hsync[c]);
-      okw = mbar_wait(&ctl.hsync[c], (n_hsync++) & 1, wc, 0x2a) && okw;
-      if (okw && q4 == 0 && lane == 0) {
-        tma_store_3d(&tm_y, half, h * kD + c * 64, (tile0 + it) * kRows, b);
+      // the 128 rows of this 64-column half are staged
+      mbar_arrive(&ctl.hsync[hf]);
+      okw = mbar_wait(&ctl.hsync[hf], (n_hsync++) & 1, wc, 0x2a) && okw;
+      if (okw && q4 == 0 && (c4 & 1) == 0 && lane == 0) {
+        tma_store_3d(&tm_y, half, h * kD + hf * 64, (tile0 + it) * kRows, b);
         bulk_commit();
         bulk_wait_read0();
         mbar_arrive(&ctl.emptyG[sg]);
@@ -474,11 +535,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       if (!ok) break;
       epilogue(it);
     }
-    if (q4 == 0 && lane == 0) bulk_wait0();
+    if (q4 == 0 && (c4 & 1) == 0 && lane == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMmaB) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
@@ -487,26 +548,35 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 constexpr size_t kStateSmem = 1024 + kStagesA * 2 * kTileB;
 constexpr size_t kOutSmem = 1024 + kTileB + kStagesQ * kTileB + kStagesG * kTileB;
 
-}  // namespace
+// The standard split of 128-dim heads (64 rotary pairs over t / h / w).
+constexpr int kStdNT = 22, kStdNH = 21;
 
-// ------------------------------------------------------------------------
-// host side
-// ------------------------------------------------------------------------
-namespace {
+bool is_std_split(const RopeDev& r) { return r.n_t == kStdNT && r.n_h == kStdNH && r.n_w == 21; }
+
+template <class K>
+void smem_attr(K kernel, size_t bytes) {
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 void set_smem_attrs() {
   static bool done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || done[dev]) return;
-  cudaFuncSetAttribute(linattn_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)(kStateSmem + kRopeSmemMax));
-  cudaFuncSetAttribute(linattn_out_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)(kOutSmem + kRopeSmemMax));
-  cudaFuncSetAttribute(linattn_out_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)(kOutSmem + kRopeSmemMax));
+  smem_attr(linattn_state_kernel<kStdNT, kStdNH>, kStateSmem + kRopeSmemMax);
+  smem_attr(linattn_state_kernel<-1, -1>, kStateSmem + kRopeSmemMax);
+  smem_attr(linattn_out_kernel<true, kStdNT, kStdNH>, kOutSmem + kRopeSmemMax);
+  smem_attr(linattn_out_kernel<false, kStdNT, kStdNH>, kOutSmem + kRopeSmemMax);
+  smem_attr(linattn_out_kernel<true, -1, -1>, kOutSmem + kRopeSmemMax);
+  smem_attr(linattn_out_kernel<false, -1, -1>, kOutSmem + kRopeSmemMax);
   done[dev] = true;
 }
+
 }  // namespace
+
+// ------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------
 
 // State phase: split reduction + fixed-order combine into S_f32 / z_out
 // (and the carried state when committing).
@@ -522,11 +592,16 @@ sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, con
     return fail(SANA_ERR_CUDA, "linattn: cuTensorMapEncodeTiled failed");
   set_smem_attrs();
   const size_t smem_a = kStateSmem + rope_smem_bytes(g, rope);
-  linattn_state_kernel<<<dim3(plan.splits_a, s.heads, s.B), kThreadsA, smem_a, st>>>(
-      tk, tv, rope, g, plan.tiles, plan.splits_a, ws_S, ws_z, status_word());
+  const dim3 grid(plan.splits_a, s.heads, s.B);
+  if (is_std_split(rope))
+    linattn_state_kernel<kStdNT, kStdNH><<<grid, kThreadsA, smem_a, st>>>(
+        tk, tv, rope, g, plan.tiles, plan.splits_a, ws_S, ws_z, status_word());
+  else
+    linattn_state_kernel<-1, -1><<<grid, kThreadsA, smem_a, st>>>(
+        tk, tv, rope, g, plan.tiles, plan.splits_a, ws_S, ws_z, status_word());
   if (sana_status e = check_launch("linattn_state_kernel")) return e;
-  linattn_combine_kernel<<<s.B * s.heads, 256, 0, st>>>(ws_S, ws_z, plan.splits_a, kD, S_prev,
-                                                        z_prev, S_state, z_state, S_f32, z_out);
+  linattn_combine_kernel<<<dim3(s.B * s.heads, kCombineSlices), 256, 0, st>>>(
+      ws_S, ws_z, plan.splits_a, kD, S_prev, z_prev, S_state, z_state, S_f32, z_out);
   return check_launch("linattn_combine_kernel");
 }
 
@@ -544,12 +619,21 @@ sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, con
   if (!okm) return fail(SANA_ERR_CUDA, "linattn: cuTensorMapEncodeTiled failed");
   set_smem_attrs();
   const size_t smem_b = kOutSmem + rope_smem_bytes(g, rope);
-  if (gt)
-    linattn_out_kernel<true><<<dim3(plan.splits_b, s.heads, s.B), kThreadsB, smem_b, st>>>(
-        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, status_word());
+  const dim3 grid(plan.splits_b, s.heads, s.B);
+  const bool stdsp = is_std_split(rope);
+  int* sw = status_word();
+  if (gt && stdsp)
+    linattn_out_kernel<true, kStdNT, kStdNH><<<grid, kThreadsB, smem_b, st>>>(
+        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
+  else if (gt)
+    linattn_out_kernel<true, -1, -1><<<grid, kThreadsB, smem_b, st>>>(
+        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
+  else if (stdsp)
+    linattn_out_kernel<false, kStdNT, kStdNH><<<grid, kThreadsB, smem_b, st>>>(
+        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
   else
-    linattn_out_kernel<false><<<dim3(plan.splits_b, s.heads, s.B), kThreadsB, smem_b, st>>>(
-        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, status_word());
+    linattn_out_kernel<false, -1, -1><<<grid, kThreadsB, smem_b, st>>>(
+        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
   return check_launch("linattn_out_kernel");
 }
 
@@ -557,8 +641,8 @@ sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, con
 void launch_linattn_combine(int BH, const float* ws_S, const float* ws_z, int splits, int D,
                             const float* S_prev, const float* z_prev, float* S_state,
                             float* z_state, float* S_f32, float* z_out, cudaStream_t st) {
-  linattn_combine_kernel<<<BH, 256, 0, st>>>(ws_S, ws_z, splits, D, S_prev, z_prev, S_state,
-                                             z_state, S_f32, z_out);
+  linattn_combine_kernel<<<dim3(BH, kCombineSlices), 256, 0, st>>>(
+      ws_S, ws_z, splits, D, S_prev, z_prev, S_state, z_state, S_f32, z_out);
 }
 
 }  // namespace sana
