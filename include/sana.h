@@ -261,6 +261,13 @@ SANA_API sana_status sana_linattn_fwd_noalloc(const sana_shape* shape, sana_dtyp
  * sana_last_error_string: thread-local message of the last non-OK status.
  * ------------------------------------------------------------------------- */
 SANA_API sana_status sana_sync_status(sana_stream_t stream);
+
+/* Failure-detection self-test: enqueues one small kernel that waits on a
+ * barrier nothing ever signals, through the same bounded wait every pipeline
+ * uses; after limit_ms (1..2000) it records a timeout in the device status word
+ * and returns normally, so the next sana_sync_status() reports SANA_ERR_TIMEOUT
+ * and the CUDA context stays usable.  No fault, trap or hang is involved. */
+SANA_API sana_status sana_selftest_bounded_wait(unsigned int limit_ms, sana_stream_t stream);
 SANA_API const char* sana_last_error_string(void);
 SANA_API const char* sana_version(void);
 

@@ -94,6 +94,7 @@ def _load():
                                           POINTER(StackWeights), POINTER(RopeStruct), c_void_p,
                                           c_void_p, c_void_p, c_size_t, c_void_p]),
         "sana_sync_status": (c_int, [c_void_p]),
+        "sana_selftest_bounded_wait": (c_int, [ctypes.c_uint, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -350,6 +351,11 @@ def hybrid_stack_fwd(x, weights, w_attn, w_ffn, rope: Rope, grid, heads, cfg: St
                                     ctypes.byref(rope.struct), _ptr(x), _ptr(out), _ptr(ws),
                                     ws.numel(), _stream()))
     return out
+
+
+def selftest_bounded_wait(limit_ms=50):
+    """Enqueue a kernel whose bounded wait runs out (see include/sana.h)."""
+    check(lib.sana_selftest_bounded_wait(limit_ms, _stream()))
 
 
 def sync_status():

@@ -48,6 +48,41 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ---- packed fp32 (f32x2) helpers: one instruction for two lanes of math
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe, for x <= 2^22 (x below -126 gives a value below
+// 2^-126, i.e. nothing in bf16).  n = round(x) comes from adding 1.5 * 2^23
+// (the low mantissa bits of the sum hold n), f = x - n lies in [-1/2, 1/2],
+// 2^f is a cubic fitted here for this interval (max relative error 7.5e-5,
+// far below bf16 rounding), and 2^n is applied by adding n to the exponent
+// field: the constant's low nine bits are zero, so the shifted sum
+// contributes exactly n << 23.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.055170517f, f, 0.24260856f), f, 0.69326097f), f, 0.99992824f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 struct AnchorCtl {
   uint64_t q_full, g_full;
   uint64_t k_full[kKS], k_empty[kKS];
@@ -58,6 +93,8 @@ struct AnchorCtl {
   int abort_flag;
 };
 
+// 320 threads = 10 warps: three share one of the four 16K-register slices of
+// the SM, which caps a thread at 168 registers.
 template <bool kGate>
 __global__ void __launch_bounds__(kThreads, 1)
     anchor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -238,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
       tmem_ld_wait();
-      float mx = -INFINITY;
       if (j == nkv - 1 && kv_tail < kRows) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -246,10 +282,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i >= kv_tail) sr[c][i] = __float_as_uint(-INFINITY);
       }
+      // row max: four independent chains of 3-input max
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+        for (int i = 0; i < 32; i += 8)
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+            mq[a] = max3(mq[a], __uint_as_float(sr[c][i + 2 * a]), __uint_as_float(sr[c][i + 2 * a + 1]));
+      const float mx = max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float m_new = fmaxf(m, mx);
       // lazy rescaling: a row moves its reference max only when the max grew
       // by more than 2^8; the decision to touch O is warp-uniform because TMEM
@@ -258,21 +300,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool any_grow = __any_sync(0xffffffffu, grow);
       const float m_use = grow ? m_new : m;
       const float corr = ex2(m - m_use);  // 0 on the first tile
-      float rs = 0.f;
+      // P = 2^(s - m): MUFU for 3 of every 4 pairs, FMA-pipe polynomial for the
+      // 4th, so the two pipes share the exponentials
+      const uint64_t neg_m = pk2(-m_use, -m_use);
+      uint64_t rs2 = pk2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2(__uint_as_float(sr[c][i]) - m_use);
-          const float p1 = ex2(__uint_as_float(sr[c][i + 1]) - m_use);
-          rs += p0 + p1;
+          float x0, x1, p0, p1;
+          up2(add2(pk2(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])), neg_m), x0, x1);
+          if ((i & 6) == 6) {
+            p0 = exp2_fma(x0);
+            p1 = exp2_fma(x1);
+          } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          rs2 = add2(rs2, pk2(p0, p1));
           pk[i / 2] = f2_to_bf2(p0, p1);
         }
         // P columns: key k lives in column k / 2 of S_i
 #pragma unroll
         for (int i = 0; i < 16; ++i) sr[c >> 1][(c & 1) * 16 + i] = pk[i];
       }
+      float rs0, rs1;
+      up2(rs2, rs0, rs1);
+      const float rs = rs0 + rs1;
       l = l * corr + rs;
       m = m_use;
       tmem_st32(tmem_s + lane_base, sr[0]);

@@ -50,6 +50,24 @@ int* status_word() {
   return addr[dev];
 }
 
+// ---------------------------------------------------------------- failure-detection self-test
+namespace {
+// Waits on an mbarrier that nothing ever arrives on, through the same bounded
+// wait every pipeline uses; after limit_ns it records a timeout and returns.
+__global__ void bounded_wait_selftest_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  const WaitCtx wc{&abort_flag, status};
+  mbar_wait(&bar, 0, wc, 0x7f, limit_ns);
+}
+}  // namespace
+
 // ---------------------------------------------------------------- tensor maps
 namespace {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -576,6 +594,15 @@ sana_status sana_gemm_bf16(long long M, int N, int K, const void* A, long long l
   if (epilogue < 0 || epilogue > 2) return fail(SANA_ERR_INVALID_ARG, "%s: bad epilogue %d", who, epilogue);
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers not 16-byte aligned", who);
   return gemm_run(M, N, K, A, lda, W, out, ldo, epilogue, stream);
+}
+
+sana_status sana_selftest_bounded_wait(unsigned int limit_ms, sana_stream_t stream) {
+  if (limit_ms == 0 || limit_ms > 2000)
+    return fail(SANA_ERR_INVALID_ARG, "sana_selftest_bounded_wait: limit_ms must be in 1..2000");
+  int* sw = status_word();
+  if (!sw) return fail(SANA_ERR_CUDA, "sana_selftest_bounded_wait: no status word on this device");
+  bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(sw, 1000000ull * limit_ms);
+  return check_launch("bounded_wait_selftest_kernel");
 }
 
 sana_status sana_sync_status(sana_stream_t stream) {

@@ -234,3 +234,20 @@ def test_causal_720p_60s_full_run():
         e = max(orc.max_rel_err(f64(y[:, rows]), yo), orc.max_rel_err(S.cpu().numpy(), So),
                 orc.max_rel_err(z.cpu().numpy(), zo))
         assert e <= BF16_TOL, (ci, e)
+
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable():
+    """A wait that can never complete gives up after its limit, the host reads
+    SANA_ERR_TIMEOUT from the device status word, and later calls work."""
+    from softmax_attention_sana_b200 import _lib as L
+    sana._lib.selftest_bounded_wait(50)
+    with pytest.raises(L.SanaError) as e:
+        sana.sync_status()
+    assert e.value.status == L.SANA_ERR_TIMEOUT
+    sana.sync_status()  # the status word was cleared
+    wl = si.TINY
+    q, k, v, g = si.qkvg(wl)
+    y = gpu_lin(q, k, v, g, (wl.T, wl.H, wl.W), wl.rope_split, wl.heads).cpu()
+    yo, _, _ = orc.linattn_bidirectional(f64(q), f64(k), f64(v), (wl.T, wl.H, wl.W),
+                                         wl.rope_split, wl.heads, gate=f64(g))
+    assert orc.max_rel_err(f64(y), yo) <= F32_TOL
