@@ -203,22 +203,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
       // O += P V: A = P in TMEM (K-major), B = V tile (MN-major: d contiguous).
       const uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
+      // operand descriptors, built once; buffers and K steps advance the address
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(q_s), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(k_s), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(v_s), kHalf, 1024);
       auto issue_s = [&](int i, int j) {  // S_i = Q'_i K'_j^T
-        const uint32_t qb = smem_u32(q_s + i * kTileB), kb = smem_u32(k_s + (j % kKS) * kTileB);
+        const uint64_t a = desc_advance(dq0, i * kTileB);
+        const uint64_t bk = desc_advance(dk0, (j % kKS) * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_ss(tmem + i * 128, smem_desc_sw128(qb + off, 16, 1024),
-                  smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk != 0);
+          umma_ss(tmem + i * 128, desc_advance(a, off), desc_advance(bk, off), idesc_s, kk != 0);
         }
         umma_commit(&ctl.s_full[i]);
       };
       auto issue_pv = [&](int i, int j) {  // O_i += P_i V_j
-        const uint32_t vb = smem_u32(v_s + (j % kVS) * kTileB);
+        const uint64_t bv = desc_advance(dv0, (j % kVS) * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk)
-          umma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8,
-                  smem_desc_sw128(vb + kk * 2048, kHalf, 1024), idesc_o, (j | kk) != 0);
+          umma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, desc_advance(bv, kk * 2048),
+                  idesc_o, (j | kk) != 0);
         umma_commit(&ctl.pv_done[i]);
       };
       bool ok = mbar_wait(&ctl.q_full, 0, wc, 0x33) && nkv > 0 &&

@@ -103,6 +103,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+      // built once; stages and K steps advance the start address
+      const uint64_t da0 = smem_desc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t db0 = smem_desc_sw128(smem_u32(smem + kABytes), 16, 1024);
       long long it = 0;
       int local = 0;
       bool ok = true;
@@ -117,11 +120,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t ab = smem_u32(smem + s * kStageBytes), bb = ab + kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma_ss(tmem + tb * BN, smem_desc_sw128(ab + kk * 32, 16, 1024),
-                    smem_desc_sw128(bb + kk * 32, 16, 1024), idesc, (kb | kk) != 0);
+            umma_ss(tmem + tb * BN, desc_advance(da0, s * kStageBytes + kk * 32),
+                    desc_advance(db0, s * kStageBytes + kk * 32), idesc, (kb | kk) != 0);
           umma_commit(&ctl.empty[s]);
         }
         if (ok) umma_commit(&ctl.tfull[tb]);

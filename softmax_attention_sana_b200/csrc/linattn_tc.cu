@@ -200,18 +200,17 @@ __global__ void __launch_bounds__(kThreadsA, 1)
       // [2 halves of 64][128 tokens]; LBO = distance of the 64-column halves,
       // SBO = distance of 8-token groups.
       const uint32_t idesc = idesc_bf16_f32(128, 128, 1, 1);
+      // built once; stages and K steps advance the start address
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(stages), kHalf, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(stages + kTileB), kHalf, 1024);
       for (int it = 0; it < ntiles; ++it) {
         const int s = it % kStagesA;
         if (!mbar_wait(&ctl.kready[s], (it / kStagesA) & 1, wc, 0x12)) break;
         tc_fence_after();
-        const uint32_t kb = smem_u32(stages + s * 2 * kTileB);
-        const uint32_t vb = kb + kTileB;
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(kb + kk * 2048, kHalf, 1024);
-          const uint64_t bd = smem_desc_sw128(vb + kk * 2048, kHalf, 1024);
-          umma_ss(tmem, ad, bd, idesc, (it | kk) != 0);
-        }
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          umma_ss(tmem, desc_advance(dk0, s * 2 * kTileB + kk * 2048),
+                  desc_advance(dv0, s * 2 * kTileB + kk * 2048), idesc, (it | kk) != 0);
         umma_commit(&ctl.empty[s]);
       }
       umma_commit(&ctl.done);
@@ -429,18 +428,18 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       // A = Q' (K-major, [2 halves][128 tok][64 d]), B = S^T (K-major,
       // [2 halves][128 e][64 d]); a K step of 16 advances 32 bytes in a half.
       const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t sb = smem_u32(s_op);
+      const uint64_t ds = smem_desc_sw128(smem_u32(s_op), 16, 1024);
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(q_st), 16, 1024);  // stages, K steps: advance
       for (int it = 0; it < ntiles; ++it) {
         const int s = it % kStagesQ, tb = it & 1;
         if (!mbar_wait(&ctl.qready[s], (it / kStagesQ) & 1, wc, 0x24)) break;
         if (it >= 2 && !mbar_wait(&ctl.tmem_free[tb], ((it >> 1) - 1) & 1, wc, 0x25)) break;
         tc_fence_after();
-        const uint32_t qb = smem_u32(q_st + s * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          umma_ss(tmem + tb * 128, smem_desc_sw128(qb + off, 16, 1024),
-                  smem_desc_sw128(sb + off, 16, 1024), idesc, kk != 0);
+          umma_ss(tmem + tb * 128, desc_advance(dq0, s * kTileB + off), desc_advance(ds, off), idesc,
+                  kk != 0);
         }
         umma_commit(&ctl.emptyQ[s]);
         umma_commit(&ctl.mma_done[tb]);

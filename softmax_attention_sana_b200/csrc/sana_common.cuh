@@ -188,6 +188,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Advance a descriptor's start address by `bytes` (a multiple of 16): the
+// start-address field sits in the low bits in 16-byte units, and shared
+// addresses stay below 2^18 bytes, so a plain add cannot carry into the next
+// field.  Lets the MMA-issuing thread build each buffer's descriptor once.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D.
 // a_mn / b_mn: operand stored MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
