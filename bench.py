@@ -293,6 +293,34 @@ def components(sana, args):
     out["causal_chunk_720p60s"] = {"ms": ms, "tokens_per_s": 10800 / (ms / 1e3),
                                    "GB_per_s": nb / (ms / 1e3) / 1e9, "l2": "flushed (256 MB) per step"}
     del q, k, v, y, flush
+    # the whole 720p/60s sequence through the block-causal scan (80 blocks of
+    # 3 frames + 1 frame, 867,600 tokens; inputs drawn on the device: 16 GB)
+    step_ms = ms
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4000)
+    shape = (1, wl.N, wl.C)
+    q, k, v = (torch.randn(shape, generator=gen, device="cuda", dtype=torch.bfloat16)
+               for _ in range(3))
+    rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
+    S = torch.zeros(1, wl.heads, wl.D, wl.D, device="cuda")
+    z = torch.zeros(1, wl.heads, wl.D, device="cuda")
+    ws = torch.empty(sana.linattn_block_causal_scan_workspace_size(1, (wl.T, wl.H, wl.W), wl.heads,
+                                                                   wl.D, 3, 1),
+                     dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(q)
+    f = lambda: sana.linattn_block_causal_scan(q, k, v, None, rope, (wl.T, wl.H, wl.W), 0,
+                                               wl.heads, 3, S, z, commit=False, out=y, ws=ws)
+    for _ in range(3):
+        f()
+    ms = time_loop(f, 10)
+    nb = 4 * wl.N * wl.C * 2 + 2 * wl.heads * (wl.D * wl.D + wl.D) * 4
+    nchunks = len(si.chunk_frames(wl))
+    out["causal_scan_720p60s"] = {
+        "ms": ms, "tokens_per_s": wl.N / (ms / 1e3), "GB_per_s": nb / (ms / 1e3) / 1e9,
+        "frac_of_hbm_peak": nb / (ms / 1e3) / 1e9 / peaks()[0],
+        "vs_chunk_steps": f"{nchunks} steps x {step_ms:.3f} ms = {nchunks * step_ms:.2f} ms",
+        "l2": "no flush: 16 GB of inputs per call"}
+    del q, k, v, y, ws
     # AttnRes route over 3 sources at 720p/5s
     srcs = [t.cuda() for t in si.attnres_sources(5, 3, 1, si.P720.N, si.P720.C)]
     w_attn, _ = (t.cuda() for t in si.router_queries(5, si.P720.C))

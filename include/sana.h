@@ -155,6 +155,34 @@ SANA_API sana_status sana_linattn_block_causal_step(const sana_shape* chunk, san
                                            sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * A whole sequence of blocks at once ([SV1] sec. 3.4 causal O_i and
+ * Algorithm 1, for rollouts whose every block is known in advance).  shape
+ * describes the sequence: T frames from absolute frame t_offset.  Block c
+ * covers frames [c * chunk_frames, (c + 1) * chunk_frames) of it; when T is
+ * not a multiple of chunk_frames the last block takes the remaining frames.
+ * The output equals running sana_linattn_block_causal_step with commit over
+ * the blocks in order from the given state (up to summation order): block c
+ * reads state_S + sum_{c' <= c} S_c'.  The blocks' own states are computed
+ * in parallel, then summed in block order (fixed order: bit-reproducible).
+ * state_S, state_z: device fp32 [B][heads][D][D] / [B][heads][D]; on entry
+ * the state before the first block (zeros = no past); commit != 0 writes the
+ * state after the last block back in place, commit == 0 leaves it untouched.
+ * chunk_frames >= 1.  Workspace: sana_linattn_block_causal_scan_workspace_size()
+ * bytes (per-block partial and prefix states, 256-byte aligned).
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_linattn_block_causal_scan_workspace_size(const sana_shape* shape,
+                                                              int chunk_frames,
+                                                              sana_dtype dtype);
+SANA_API sana_status sana_linattn_block_causal_scan(const sana_shape* shape, int chunk_frames,
+                                                    sana_dtype dtype, const void* q,
+                                                    const void* k, const void* v,
+                                                    const void* gate_logits,
+                                                    const sana_rope* rope, float eps,
+                                                    float* state_S, float* state_z, int commit,
+                                                    void* out, void* ws, size_t ws_bytes,
+                                                    sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Gated softmax anchor ([SV2a]; reading: the same 3D RoPE on raw Q, K):
  *   Y = sigmoid(G) * softmax(RoPE(Q) RoPE(K)^T * scale) V, bidirectional over
  *   all N keys of the same batch entry and head.

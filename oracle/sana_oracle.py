@@ -220,6 +220,37 @@ def linattn_block_causal_step(q, k, v, chunk_grid, t_offset, rope_split, heads,
     return y, np.array(S_prev, np.float64), np.array(z_prev, np.float64)
 
 
+def linattn_block_causal_sequence(q, k, v, grid, chunk_frames, t_offset, rope_split, heads,
+                                  S_prev, z_prev, gate=None, eps=EPS, commit=True):
+    """A whole sequence of blocks ([SV1] sec. 3.4, Algorithm 1), each of
+    `chunk_frames` frames except a shorter last block when the frame count is
+    not a multiple of it (reading: the remainder forms the final block).
+
+    The blocks go through linattn_block_causal_step in order, each committing
+    its contribution so that the next block sees it; with commit the state
+    after the last block is returned, otherwise the initial state.
+    Returns (Y, S, z)."""
+    T, H, W = grid
+    hw = H * W
+    S = np.asarray(S_prev, np.float64)
+    z = np.asarray(z_prev, np.float64)
+    ys = []
+    t0 = 0
+    while t0 < T:
+        f = min(chunk_frames, T - t0)
+        sl = slice(t0 * hw, (t0 + f) * hw)
+        y, S, z = linattn_block_causal_step(
+            q[:, sl], k[:, sl], v[:, sl], (f, H, W), t_offset + t0, rope_split, heads, S, z,
+            gate=None if gate is None else gate[:, sl], eps=eps, commit=True)
+        ys.append(y)
+        t0 += f
+    B, _, C = np.asarray(v).shape
+    y = np.concatenate(ys, axis=1) if ys else np.zeros((B, 0, C))
+    if commit:
+        return y, S, z
+    return y, np.array(S_prev, np.float64), np.array(z_prev, np.float64)
+
+
 def linattn_token_recurrence(q, k, v, grid, rope_split, heads, eps=EPS):
     """Per-token causal recurrence of [SV1] sec. 3.4 (chunk size 1), with RoPE
     in the numerator: O_i = RoPE(phi Q_i)(sum_{j<i} S_j + S_i) / (phi Q_i (sum_{j<=i} phi K_j) + eps)."""

@@ -80,6 +80,11 @@ def _load():
                                                    c_void_p, c_void_p, POINTER(RopeStruct), c_float,
                                                    c_void_p, c_void_p, c_int, c_void_p, c_void_p,
                                                    c_size_t, c_void_p]),
+        "sana_linattn_block_causal_scan_workspace_size": (c_size_t, [POINTER(Shape), c_int, c_int]),
+        "sana_linattn_block_causal_scan": (c_int, [POINTER(Shape), c_int, c_int, c_void_p, c_void_p,
+                                                   c_void_p, c_void_p, POINTER(RopeStruct),
+                                                   c_float, c_void_p, c_void_p, c_int, c_void_p,
+                                                   c_void_p, c_size_t, c_void_p]),
         "sana_softmax_anchor_workspace_size": (c_size_t, [POINTER(Shape), c_int]),
         "sana_softmax_anchor_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, POINTER(RopeStruct), c_float, c_void_p,
@@ -253,6 +258,35 @@ def linattn_block_causal_step(q, k, v, gate, rope: Rope, grid, t_offset, heads, 
     check(lib.sana_linattn_block_causal_step(
         ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(rope.struct), eps,
         _ptr(state_S), _ptr(state_z), int(bool(commit)), _ptr(out), _ptr(ws), ws.numel(), _stream()))
+    return out
+
+
+def linattn_block_causal_scan_workspace_size(B, grid, heads, D, chunk_frames, dtype_code,
+                                             t_offset=0) -> int:
+    s = make_shape(B, grid, heads, D, t_offset)
+    return lib.sana_linattn_block_causal_scan_workspace_size(ctypes.byref(s), chunk_frames,
+                                                             dtype_code)
+
+
+def linattn_block_causal_scan(q, k, v, gate, rope: Rope, grid, t_offset, heads, chunk_frames,
+                              state_S, state_z, commit=True, eps=1e-6, out=None, ws=None):
+    """A whole sequence of blocks of chunk_frames frames (the last block takes the
+    remaining frames); state_S / state_z fp32 in place as for the block step."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (state_S, "state_S"), (state_z, "state_z")):
+        _need(t, n)
+    B, N, C = q.shape
+    D = C // heads
+    dt = _dtype_code(q)
+    s = make_shape(B, grid, heads, D, t_offset)
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = _ws(lib.sana_linattn_block_causal_scan_workspace_size(ctypes.byref(s), chunk_frames,
+                                                                   dt), q.device)
+    check(lib.sana_linattn_block_causal_scan(
+        ctypes.byref(s), chunk_frames, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
+        ctypes.byref(rope.struct), eps, _ptr(state_S), _ptr(state_z), int(bool(commit)), _ptr(out),
+        _ptr(ws), ws.numel(), _stream()))
     return out
 
 

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     tmem_alloc(&ctl.tmem, 128);
     tmem_relinquish();
   }
-  const RopeSmem rs = rope_stage(rope_base, rope, g, tid, kThreadsA);
+  const RopeSmem rs = rope_stage(rope_base, rope, g, b, tid, kThreadsA);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
     fence_proxy_async_smem();
   }
-  const RopeSmem rs = rope_stage(rope_base, rope, g, tid, kThreadsB);
+  const RopeSmem rs = rope_stage(rope_base, rope, g, b, tid, kThreadsB);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -577,13 +577,11 @@ void set_smem_attrs() {
 // host side
 // ------------------------------------------------------------------------
 
-// State phase: split reduction + fixed-order combine into S_f32 / z_out
-// (and the carried state when committing).
-sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, const void* k,
-                               const void* v, const RopeDev& rope, const GridDev& g,
-                               const float* S_prev, const float* z_prev, float* S_state,
-                               float* z_state, float* ws_S, float* ws_z, float* S_f32,
-                               float* z_out, cudaStream_t st) {
+// Split reduction only: partial S and z of every (batch entry, head, split)
+// into ws_S [B][heads][splits][D][D] and ws_z [B][heads][splits][D].
+sana_status linattn_bf16_partials(const sana_shape& s, const LinAttnPlan& plan, const void* k,
+                                  const void* v, const RopeDev& rope, const GridDev& g,
+                                  float* ws_S, float* ws_z, cudaStream_t st) {
   const uint64_t C = (uint64_t)s.heads * kD, N = (uint64_t)g.N;
   CUtensorMap tk, tv;
   if (!make_tmap_bf16_3d(&tk, k, C, N, s.B, C, N * C, kRows) ||
@@ -598,7 +596,17 @@ sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, con
   else
     linattn_state_kernel<-1, -1><<<grid, kThreadsA, smem_a, st>>>(
         tk, tv, rope, g, plan.tiles, plan.splits_a, ws_S, ws_z, status_word());
-  if (sana_status e = check_launch("linattn_state_kernel")) return e;
+  return check_launch("linattn_state_kernel");
+}
+
+// State phase: split reduction + fixed-order combine into S_f32 / z_out
+// (and the carried state when committing).
+sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, const void* k,
+                               const void* v, const RopeDev& rope, const GridDev& g,
+                               const float* S_prev, const float* z_prev, float* S_state,
+                               float* z_state, float* ws_S, float* ws_z, float* S_f32,
+                               float* z_out, cudaStream_t st) {
+  if (sana_status e = linattn_bf16_partials(s, plan, k, v, rope, g, ws_S, ws_z, st)) return e;
   linattn_combine_kernel<<<dim3(s.B * s.heads, kCombineSlices), 256, 0, st>>>(
       ws_S, ws_z, plan.splits_a, kD, S_prev, z_prev, S_state, z_state, S_f32, z_out);
   return check_launch("linattn_combine_kernel");

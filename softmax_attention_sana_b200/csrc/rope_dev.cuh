@@ -22,9 +22,10 @@ struct RopeSmem {
 
 __device__ __forceinline__ int odd_up_d(int n) { return n | 1; }
 
-// Cooperative staging by `nthreads` threads; caller synchronises afterwards.
-__device__ inline RopeSmem rope_stage(float2* base, const RopeDev& r, const GridDev& g, int tid,
-                                      int nthreads) {
+// Cooperative staging by `nthreads` threads for batch entry b; caller
+// synchronises afterwards.
+__device__ inline RopeSmem rope_stage(float2* base, const RopeDev& r, const GridDev& g, int b,
+                                      int tid, int nthreads) {
   RopeSmem rs;
   rs.st = odd_up_d(r.n_t);
   rs.sh = odd_up_d(r.n_h);
@@ -34,7 +35,7 @@ __device__ inline RopeSmem rope_stage(float2* base, const RopeDev& r, const Grid
   float2* pw = ph + g.H * rs.sh;
   for (int i = tid; i < g.T * r.n_t; i += nthreads) {
     const int row = i / r.n_t, j = i - row * r.n_t;
-    const int src = (g.t_offset + row) * r.n_t + j;
+    const int src = (g.t_offset + b * g.t_stride + row) * r.n_t + j;
     pt[row * rs.st + j] = make_float2(r.cos_t[src], r.sin_t[src]);
   }
   for (int i = tid; i < g.H * r.n_h; i += nthreads) {
@@ -79,15 +80,16 @@ __device__ __forceinline__ RowRope row_rope(const RopeSmem& rs, const GridDev& g
   return rr;
 }
 
-// Same lookup straight from the global tables (fp32 paths).
-__device__ __forceinline__ float2 rope_cs_global(const RopeDev& r, const GridDev& g, int n, int j) {
+// Same lookup straight from the global tables (fp32 paths), batch entry b.
+__device__ __forceinline__ float2 rope_cs_global(const RopeDev& r, const GridDev& g, int b, int n,
+                                                 int j) {
   const int hw = g.H * g.W;
   const int t = n / hw;
   const int rem = n - t * hw;
   const int h = rem / g.W;
   const int w = rem - h * g.W;
   if (j < r.n_t) {
-    const int i = (g.t_offset + t) * r.n_t + j;
+    const int i = (g.t_offset + b * g.t_stride + t) * r.n_t + j;
     return make_float2(r.cos_t[i], r.sin_t[i]);
   }
   if (j < r.n_t + r.n_h) {

@@ -167,25 +167,6 @@ GridDev to_grid(const sana_shape& s) {
 }  // namespace
 
 // ---------------------------------------------------------------- linear attention
-sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, const void* k,
-                               const void* v, const RopeDev& rope, const GridDev& g,
-                               const float* S_prev, const float* z_prev, float* S_state,
-                               float* z_state, float* ws_S, float* ws_z, float* S_f32,
-                               float* z_out, cudaStream_t st);
-sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, const void* q,
-                               const void* gt, const RopeDev& rope, const GridDev& g,
-                               const float* S_f32, const float* z, float eps, void* out,
-                               cudaStream_t st);
-int linattn_f32_splits(const sana_shape& s, int N);
-sana_status linattn_f32_state(const sana_shape& s, const float* k, const float* v,
-                              const RopeDev& rope, const GridDev& g, int splits,
-                              const float* S_prev, const float* z_prev, float* S_state,
-                              float* z_state, float* ws_S, float* ws_z, float* S_f32,
-                              float* z_comb, cudaStream_t st);
-sana_status linattn_f32_apply(const sana_shape& s, const float* q, const float* gt,
-                              const RopeDev& rope, const GridDev& g, const float* S_f32,
-                              const float* z, float eps, float* out, cudaStream_t st);
-
 LinAttnPlan linattn_plan(const sana_shape& s, sana_dtype dt) {
   LinAttnPlan p{};
   const int N = s.T * s.H * s.W;
@@ -470,6 +451,49 @@ sana_status sana_linattn_block_causal_step(const sana_shape* s, sana_dtype dt, c
                                            sana_stream_t stream) {
   return linattn_common("sana_linattn_block_causal_step", s, dt, q, k, v, g, rope, eps, S, z, true,
                         commit, out, ws, ws_bytes, stream);
+}
+
+size_t sana_linattn_block_causal_scan_workspace_size(const sana_shape* s, int chunk_frames,
+                                                     sana_dtype dt) {
+  if (check_shape(s, dt, "sana_linattn_block_causal_scan_workspace_size") != SANA_OK ||
+      chunk_frames < 1)
+    return 0;
+  return linattn_scan_ws_bytes(*s, chunk_frames, dt);
+}
+
+sana_status sana_linattn_block_causal_scan(const sana_shape* s, int chunk_frames, sana_dtype dt,
+                                           const void* q, const void* k, const void* v,
+                                           const void* g, const sana_rope* rope, float eps,
+                                           float* S, float* z, int commit, void* out, void* ws,
+                                           size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_linattn_block_causal_scan";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (sana_status e = check_rope(rope, s, who)) return e;
+  if (chunk_frames < 1) return fail(SANA_ERR_INVALID_ARG, "%s: chunk_frames=%d", who, chunk_frames);
+  if (!std::isfinite(eps) || eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", who);
+  if (!S || !z) return fail(SANA_ERR_INVALID_ARG, "%s: state pointers are NULL", who);
+  if (!aligned16(S) || !aligned16(z)) return fail(SANA_ERR_INVALID_ARG, "%s: state must be 16-byte aligned", who);
+  if (s->T == 0) return SANA_OK;  // no blocks: nothing to read or write, state unchanged
+  if (!q || !k || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  const void* ptrs[5] = {q, k, v, g, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
+  if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, g, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an input", who);
+  const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
+  const size_t zb = (size_t)s->B * s->heads * s->head_dim * 4;
+  if (overlap(S, sb, out, n) || overlap(z, zb, out, n) || overlap(S, sb, z, zb))
+    return fail(SANA_ERR_INVALID_ARG, "%s: state aliases the output", who);
+  const size_t need = linattn_scan_ws_bytes(*s, chunk_frames, dt);
+  if (!ws || ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  if (overlap(ws, need, out, n) || overlap(ws, need, S, sb) || overlap(ws, need, z, zb))
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace aliases the output or the state", who);
+  return linattn_scan_run(*s, chunk_frames, dt, q, k, v, g, to_dev(*rope), eps, S, z, commit != 0,
+                          out, ws, ws_bytes, stream);
 }
 
 size_t sana_linattn_state_workspace_size(const sana_shape* s, sana_dtype dt) {

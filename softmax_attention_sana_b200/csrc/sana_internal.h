@@ -50,12 +50,15 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                        uint64_t row_stride, uint32_t box_cols, uint32_t box_rows);
 
-// Grid of one call, as the kernels see it.
+// Grid of one call, as the kernels see it.  Batch entry b covers frames
+// [t_offset + b * t_stride, + T): t_stride is 0 for independent sequences and
+// the block length when consecutive blocks of one sequence are batched.
 struct GridDev {
   int T, H, W;
   int t_offset;
   int N;
   int heads;
+  int t_stride = 0;
 };
 // RoPE tables, as the kernels see them.
 struct RopeDev {
@@ -87,11 +90,49 @@ sana_status linattn_apply_run(const sana_shape& s, sana_dtype dt, const void* q,
                               const RopeDev& rope, const float* S, const float* z, float eps,
                               void* out, cudaStream_t st);
 
+// Launchers of the two precisions (linattn_tc.cu for bf16, simt_f32.cu for fp32).
+// The partial launchers run the split reduction only; ws_S / ws_z receive
+// [B][heads][splits][D][D] / [B][heads][splits][D].
+sana_status linattn_bf16_partials(const sana_shape& s, const LinAttnPlan& plan, const void* k,
+                                  const void* v, const RopeDev& rope, const GridDev& g,
+                                  float* ws_S, float* ws_z, cudaStream_t st);
+sana_status linattn_f32_partials(const sana_shape& s, const float* k, const float* v,
+                                 const RopeDev& rope, const GridDev& g, int splits, float* ws_S,
+                                 float* ws_z, cudaStream_t st);
+sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, const void* k,
+                               const void* v, const RopeDev& rope, const GridDev& g,
+                               const float* S_prev, const float* z_prev, float* S_state,
+                               float* z_state, float* ws_S, float* ws_z, float* S_f32,
+                               float* z_out, cudaStream_t st);
+sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, const void* q,
+                               const void* gt, const RopeDev& rope, const GridDev& g,
+                               const float* S_f32, const float* z, float eps, void* out,
+                               cudaStream_t st);
+int linattn_f32_splits(const sana_shape& s, int N);
+sana_status linattn_f32_state(const sana_shape& s, const float* k, const float* v,
+                              const RopeDev& rope, const GridDev& g, int splits,
+                              const float* S_prev, const float* z_prev, float* S_state,
+                              float* z_state, float* ws_S, float* ws_z, float* S_f32,
+                              float* z_comb, cudaStream_t st);
+sana_status linattn_f32_apply(const sana_shape& s, const float* q, const float* gt,
+                              const RopeDev& rope, const GridDev& g, const float* S_f32,
+                              const float* z, float eps, float* out, cudaStream_t st);
+
+
 // Bidirectional (S_prev == nullptr) or block-causal step.
 sana_status linattn_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,
                         const void* v, const void* g, const RopeDev& rope, float eps,
                         float* state_S, float* state_z, bool causal, bool commit, void* out,
                         void* ws, size_t ws_bytes, cudaStream_t st);
+
+// A whole sequence of blocks of `chunk_frames` frames (the last block takes
+// the remaining frames): per-block states in parallel, a fixed-order prefix
+// over blocks, then every block's output.
+size_t linattn_scan_ws_bytes(const sana_shape& s, int chunk_frames, sana_dtype dt);
+sana_status linattn_scan_run(const sana_shape& s, int chunk_frames, sana_dtype dt, const void* q,
+                             const void* k, const void* v, const void* g, const RopeDev& rope,
+                             float eps, float* state_S, float* state_z, bool commit, void* out,
+                             void* ws, size_t ws_bytes, cudaStream_t st);
 
 // ---------------------------------------------------------------- softmax anchor
 size_t anchor_ws_bytes(const sana_shape& s, sana_dtype dt);

@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(256)
       }
       kphi[tok][2 * j] = x;
       kphi[tok][2 * j + 1] = y;
-      const float2 r = n < g.N ? rotate(x, y, rope_cs_global(rope, g, n, j)) : make_float2(0.f, 0.f);
+      const float2 r = n < g.N ? rotate(x, y, rope_cs_global(rope, g, b, n, j)) : make_float2(0.f, 0.f);
       kp[tok][2 * j] = r.x;
       kp[tok][2 * j + 1] = r.y;
       vs[tok][2 * j] = vx;
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(256)
     }
     qphi[tok * D + 2 * j] = x;
     qphi[tok * D + 2 * j + 1] = yv;
-    const float2 r = n < g.N ? rotate(x, yv, rope_cs_global(rope, g, n, j)) : make_float2(0.f, 0.f);
+    const float2 r = n < g.N ? rotate(x, yv, rope_cs_global(rope, g, b, n, j)) : make_float2(0.f, 0.f);
     qp[tok * D + 2 * j] = r.x;
     qp[tok * D + 2 * j + 1] = r.y;
   }
@@ -150,7 +150,7 @@ __global__ void rope_rotate_kernel(const T* __restrict__ x, RopeDev rope, GridDe
       a = __bfloat162float(x[off]);
       c = __bfloat162float(x[off + 1]);
     }
-    float2 r = rope.cos_t ? rotate(a, c, rope_cs_global(rope, g, n, j)) : make_float2(a, c);
+    float2 r = rope.cos_t ? rotate(a, c, rope_cs_global(rope, g, b, n, j)) : make_float2(a, c);
     r.x *= mul;
     r.y *= mul;
     if constexpr (sizeof(T) == 4) {
@@ -216,12 +216,18 @@ __global__ void __launch_bounds__(128)
 }
 
 template <int D>
+void run_partials(const sana_shape& s, const float* k, const float* v, const RopeDev& rope,
+                  const GridDev& g, int splits, float* ws_S, float* ws_z, cudaStream_t st) {
+  linattn_state_f32_kernel<D><<<dim3(splits, s.heads, s.B), 256, 0, st>>>(k, v, rope, g, splits,
+                                                                          ws_S, ws_z);
+}
+
+template <int D>
 void run_state(const sana_shape& s, const float* k, const float* v, const RopeDev& rope,
                const GridDev& g, int splits, const float* S_prev, const float* z_prev,
                float* S_state, float* z_state, float* ws_S, float* ws_z, float* S_f32,
                float* z_comb, cudaStream_t st) {
-  linattn_state_f32_kernel<D><<<dim3(splits, s.heads, s.B), 256, 0, st>>>(k, v, rope, g, splits,
-                                                                          ws_S, ws_z);
+  run_partials<D>(s, k, v, rope, g, splits, ws_S, ws_z, st);
   launch_linattn_combine(s.B * s.heads, ws_S, ws_z, splits, D, S_prev, z_prev, S_state, z_state,
                          S_f32, z_comb, st);
 }
@@ -267,6 +273,19 @@ sana_status linattn_f32_state(const sana_shape& s, const float* k, const float* 
     default: return fail(SANA_ERR_UNSUPPORTED, "fp32 linear attention: head_dim %d", s.head_dim);
   }
   return check_launch("linattn fp32 state kernels");
+}
+
+sana_status linattn_f32_partials(const sana_shape& s, const float* k, const float* v,
+                                 const RopeDev& rope, const GridDev& g, int splits, float* ws_S,
+                                 float* ws_z, cudaStream_t st) {
+  switch (s.head_dim) {
+    case 16: run_partials<16>(s, k, v, rope, g, splits, ws_S, ws_z, st); break;
+    case 32: run_partials<32>(s, k, v, rope, g, splits, ws_S, ws_z, st); break;
+    case 64: run_partials<64>(s, k, v, rope, g, splits, ws_S, ws_z, st); break;
+    case 128: run_partials<128>(s, k, v, rope, g, splits, ws_S, ws_z, st); break;
+    default: return fail(SANA_ERR_UNSUPPORTED, "fp32 linear attention: head_dim %d", s.head_dim);
+  }
+  return check_launch("linattn_state_f32_kernel");
 }
 
 sana_status linattn_f32_apply(const sana_shape& s, const float* q, const float* gt,

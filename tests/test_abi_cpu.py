@@ -111,6 +111,33 @@ def test_validation_errors_return_before_any_device_work():
     assert st == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
 
 
+def _call_scan(shape, frames, S=8 << 20, z=9 << 20, ws_bytes=1 << 24, out=4 << 20):
+    # fake device addresses, 1 MiB apart: every call here fails validation first
+    r = _lib.RopeStruct(16, 16, 16, 16, 16, 16, 2, 3, 3, 8, 4, 4)
+    return _lib.lib.sana_linattn_block_causal_scan(
+        ctypes.byref(shape), frames, _lib.SANA_F32, 1 << 20, 2 << 20, 3 << 20, None,
+        ctypes.byref(r), 1e-6, S, z, 1, out, 1 << 26, ws_bytes, None)
+
+
+def test_block_causal_scan_sizes_and_validation():
+    L = _lib
+    # 720p/60s: 80 blocks of 3 frames (one split each: 80 x 24 CTAs fill the
+    # GPU) + a 1-frame block (148 // 24 = 6 splits), then 81 prefix states
+    long_seq = _shape(T=241, H=45, W=80, heads=24, head_dim=128)
+    ws = L.lib.sana_linattn_block_causal_scan_workspace_size(ctypes.byref(long_seq), 3, L.SANA_BF16)
+    per_state = 24 * (128 * 128 + 128) * 4
+    want = (80 + 6 + 81) * per_state
+    assert want <= ws < want + 8 * 256
+    assert L.lib.sana_linattn_block_causal_scan_workspace_size(ctypes.byref(long_seq), 0,
+                                                               L.SANA_BF16) == 0
+    s = _shape(T=8)
+    assert _call_scan(s, 0) == L.SANA_ERR_INVALID_ARG and "chunk_frames" in L.last_error()
+    assert _call_scan(s, 3, S=None) == L.SANA_ERR_INVALID_ARG
+    assert _call_scan(s, 3, S=(8 << 20) + 4) == L.SANA_ERR_INVALID_ARG
+    assert _call_scan(s, 3, ws_bytes=64) == L.SANA_ERR_WORKSPACE
+    assert _call_scan(s, 3, out=2 << 20) == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
+
+
 def test_attnres_and_gemm_validation():
     L = _lib
     arr = (ctypes.c_void_p * 1)(4096)

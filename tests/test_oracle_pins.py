@@ -211,6 +211,46 @@ def test_chunked_equals_masked_bruteforce(chunks):
     assert rel(y, yb) < 1e-12
 
 
+@pytest.mark.parametrize("frames", [1, 2, 3, 4, 7, 9])
+def test_block_sequence_equals_masked_bruteforce(frames):
+    """A whole sequence in blocks of `frames` frames (7 = 3 + 3 + 1 for
+    frames=3, one block when frames >= 7): brute force with chunk(j) <= chunk(i)."""
+    grid, split, heads = (7, 2, 3), (2, 1, 1), 2
+    T = grid[0]
+    N = T * 6
+    q, k, v, g = _lin_inputs(1, N, heads, 8)
+    S0, z0 = np.zeros((1, heads, 8, 8)), np.zeros((1, heads, 8))
+    y, S, z = orc.linattn_block_causal_sequence(q, k, v, grid, frames, 0, split, heads, S0, z0,
+                                                gate=g)
+    sizes = [min(frames, T - t) for t in range(0, T, frames)]
+    yb = orc.linattn_bruteforce(q, k, v, grid, split, heads, gate=g, mask=_frame_mask(grid, sizes))
+    assert rel(y, yb) < 1e-12
+    _, S_bi, z_bi = orc.linattn_bidirectional(q, k, v, grid, split, heads, gate=g)
+    assert rel(S, S_bi) < 1e-13 and rel(z, z_bi) < 1e-13
+
+
+def test_block_sequence_resumes_from_a_carried_state():
+    """Frames [0, 4) then [4, 7) from the carried state (absolute frames from
+    t_offset = 4) equal the whole sequence; without commit the state is kept."""
+    grid, split, heads = (7, 2, 3), (2, 1, 1), 2
+    hw = 6
+    q, k, v, g = _lin_inputs(2, 7 * hw, heads, 8)
+    S0, z0 = np.zeros((2, heads, 8, 8)), np.zeros((2, heads, 8))
+    y_all, S_all, z_all = orc.linattn_block_causal_sequence(q, k, v, grid, 2, 0, split, heads,
+                                                            S0, z0, gate=g)
+    a, r = slice(0, 4 * hw), slice(4 * hw, 7 * hw)
+    y_a, S_a, z_a = orc.linattn_block_causal_sequence(q[:, a], k[:, a], v[:, a], (4, 2, 3), 2, 0,
+                                                      split, heads, S0, z0, gate=g[:, a])
+    y_r, S_r, z_r = orc.linattn_block_causal_sequence(q[:, r], k[:, r], v[:, r], (3, 2, 3), 2, 4,
+                                                      split, heads, S_a, z_a, gate=g[:, r])
+    assert rel(np.concatenate([y_a, y_r], axis=1), y_all) < 1e-13
+    assert rel(S_r, S_all) < 1e-13 and rel(z_r, z_all) < 1e-13
+    y_n, S_n, z_n = orc.linattn_block_causal_sequence(q[:, r], k[:, r], v[:, r], (3, 2, 3), 2, 4,
+                                                      split, heads, S_a, z_a, gate=g[:, r],
+                                                      commit=False)
+    assert rel(y_n, y_r) == 0 and np.array_equal(S_n, S_a) and np.array_equal(z_n, z_a)
+
+
 def test_token_recurrence_equals_prefix_recomputation():
     """Chunk size 1 token: the sec. 3.4 recurrence = brute force with j <= i."""
     grid, split, heads = (2, 3, 4), (2, 1, 1), 2
