@@ -36,6 +36,9 @@ constexpr int kVS = 2;                 // V stages
 constexpr int kThreads = 320;          // 8 softmax warps + producer + MMA
 constexpr int kWarpProd = 8, kWarpMma = 9;
 constexpr float kRescaleLog2 = 8.f;    // lazy rescale threshold (base-2 units)
+// Of every 8 pairs of exponentials, this many run as a polynomial on the FMA
+// pipe instead of the MUFU unit (16 results per clock per SM).
+constexpr int kEmuPairs = 2;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -62,6 +65,16 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -75,12 +88,27 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // far below bf16 rounding), and 2^n is applied by adding n to the exponent
 // field: the constant's low nine bits are zero, so the shifted sum
 // contributes exactly n << 23.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.055170517f, f, 0.24260856f), f, 0.69326097f), f, 0.99992824f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+//
+// Two at a time with packed f32x2 arithmetic, with the max subtraction folded
+// in: for a row with reference max m, x = s - m; c = 1.5 * 2^23 - m gives
+// t = s + c = round(x) + 1.5 * 2^23 and f = s - (t - c) = x - round(x).
+// s_lo = m - 126 is the clamp; the exponent add is one integer multiply-add.
+__device__ __forceinline__ void exp2_fma2(float s0, float s1, float s_lo, uint64_t c,
+                                          float& y0, float& y1) {
+  const uint64_t sv = pk2(fmaxf(s0, s_lo), fmaxf(s1, s_lo));
+  const uint64_t t = add2(sv, c);
+  const uint64_t f = sub2(sv, sub2(t, c));
+  uint64_t p = fma2(pk2(0.055170517f, 0.055170517f), f, pk2(0.24260856f, 0.24260856f));
+  p = fma2(p, f, pk2(0.69326097f, 0.69326097f));
+  p = fma2(p, f, pk2(0.99992824f, 0.99992824f));
+  float t0, t1, p0, p1;
+  up2(t, t0, t1);
+  up2(p, p0, p1);
+  uint32_t r0, r1;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(p0)));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(__float_as_uint(t1)), "r"(__float_as_uint(p1)));
+  y0 = __uint_as_float(r0);
+  y1 = __uint_as_float(r1);
 }
 
 struct AnchorCtl {
@@ -275,67 +303,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
-      tmem_ld_wait();
-      if (j == nkv - 1 && kv_tail < kRows) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i >= kv_tail) sr[c][i] = __float_as_uint(-INFINITY);
-      }
-      // row max: four independent chains of 3-input max
+      const bool last = j == nkv - 1 && kv_tail < kRows;
+      // pass 1: row max, 64 columns in registers at a time (four independent
+      // chains of 3-input max)
       float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tmem_s + lane_base + hh * 64, sa);
+        tmem_ld32(tmem_s + lane_base + hh * 64 + 32, sb);
+        tmem_ld_wait();
+        if (last) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (hh * 64 + i >= kv_tail) sa[i] = __float_as_uint(-INFINITY);
+            if (hh * 64 + 32 + i >= kv_tail) sb[i] = __float_as_uint(-INFINITY);
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 32; i += 8)
 #pragma unroll
           for (int a = 0; a < 4; ++a)
-            mq[a] = max3(mq[a], __uint_as_float(sr[c][i + 2 * a]), __uint_as_float(sr[c][i + 2 * a + 1]));
+            mq[a] = max3(mq[a], __uint_as_float(sa[i + 2 * a]), __uint_as_float(sb[i + 2 * a + 1]));
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+            mq[a] = max3(mq[a], __uint_as_float(sa[i + 2 * a + 1]), __uint_as_float(sb[i + 2 * a]));
+      }
       const float mx = max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float m_new = fmaxf(m, mx);
       // lazy rescaling: a row moves its reference max only when the max grew
       // by more than 2^8; the decision to touch O is warp-uniform because TMEM
-      // access is warp-collective (rows that keep their max use a factor 1)
+      // access is warp-collective (rows that keep their max use a factor 1).
+      // A moved max is rounded up to an integer so that the folded constant of
+      // the FMA-pipe exponential (1.5 * 2^23 - m) is exact.
       const bool grow = m_new > m + kRescaleLog2;
       const bool any_grow = __any_sync(0xffffffffu, grow);
-      const float m_use = grow ? m_new : m;
+      const float m_use = grow ? ceilf(m_new) : m;
       const float corr = ex2(m - m_use);  // 0 on the first tile
-      // P = 2^(s - m): MUFU for 3 of every 4 pairs, FMA-pipe polynomial for the
-      // 4th, so the two pipes share the exponentials
+      // pass 2: P = 2^(s - m) over 32-column chunks, the next chunk's load in
+      // flight while this one is exponentiated (MUFU for most pairs, the
+      // FMA-pipe polynomial for kEmuPairs of every 8).  P of chunk c goes to
+      // columns [16c, 16c + 16), inside S chunks already read.
       const uint64_t neg_m = pk2(-m_use, -m_use);
+      const uint64_t cfold = pk2(12582912.f - m_use, 12582912.f - m_use);
+      const float s_lo = m_use - 126.f;
       uint64_t rs2 = pk2(0.f, 0.f);
+      uint32_t sc[2][32];
+      uint32_t pk[32];
+      tmem_ld32(tmem_s + lane_base, sc[0]);
+      tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        if (c < 3) tmem_ld32(tmem_s + lane_base + (c + 1) * 32, sc[(c + 1) & 1]);
+        uint32_t* cur = sc[c & 1];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float x0, x1, p0, p1;
-          up2(add2(pk2(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])), neg_m), x0, x1);
-          if ((i & 6) == 6) {
-            p0 = exp2_fma(x0);
-            p1 = exp2_fma(x1);
+          float s0 = __uint_as_float(cur[i]), s1 = __uint_as_float(cur[i + 1]);
+          if (last) {
+            if (c * 32 + i >= kv_tail) s0 = -INFINITY;
+            if (c * 32 + i + 1 >= kv_tail) s1 = -INFINITY;
+          }
+          float p0, p1;
+          if (((i >> 1) & 7) >= 8 - kEmuPairs) {
+            exp2_fma2(s0, s1, s_lo, cfold, p0, p1);
           } else {
+            float x0, x1;
+            up2(add2(pk2(s0, s1), neg_m), x0, x1);
             p0 = ex2(x0);
             p1 = ex2(x1);
           }
           rs2 = add2(rs2, pk2(p0, p1));
-          pk[i / 2] = f2_to_bf2(p0, p1);
+          pk[(c & 1) * 16 + i / 2] = f2_to_bf2(p0, p1);
         }
-        // P columns: key k lives in column k / 2 of S_i
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sr[c >> 1][(c & 1) * 16 + i] = pk[i];
+        if (c & 1) tmem_st32(tmem_s + lane_base + (c >> 1) * 32, pk);
+        if (c < 3) tmem_ld_wait();
       }
       float rs0, rs1;
       up2(rs2, rs0, rs1);
-      const float rs = rs0 + rs1;
-      l = l * corr + rs;
+      l = l * corr + (rs0 + rs1);
       m = m_use;
-      tmem_st32(tmem_s + lane_base, sr[0]);
-      tmem_st32(tmem_s + lane_base + 32, sr[1]);
       if (any_grow && j >= 1) {
         // O_i holds the sum over tiles < j (their PV MMAs finished before S_i
         // of this tile was issued); scale it before the next PV accumulates
