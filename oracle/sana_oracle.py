@@ -45,12 +45,19 @@ Readings where the pages are silent (each also listed in the design doc):
   left out while it is empty.
 * Stack: layer l is an anchor iff l % 4 == 3; FFN = W_down SiLU(W_up x) with
   hidden size ffn_mult * C; sublayer input RMSNorm(h) without gain.
+* Sparse anchor ([SV2] Experiments and [SV2-abs] say only that the
+  deployment stack applies sparse attention to the softmax anchors): queries
+  in blocks of 256 tokens, keys in tiles of 128; each block keeps the `keep`
+  key tiles with the largest pooled logit mean(RoPE(Q) * scale) .
+  mean(RoPE(K)) (ties to the lower tile index) and attends to exactly those
+  keys.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 against brute force, closed forms or invariants, except the absolute values
 that only the readings above fix (RoPE layout and frequencies, eps values,
 the anchor's use of RoPE, the FFN form, the empty-partial-sum and last-chunk
-rules): those are "parity unpinned" beyond the readings themselves.
+rules, and the whole block-sparse pattern of the sparse anchor): those are
+"parity unpinned" beyond the readings themselves.
 """
 
 from __future__ import annotations
@@ -307,6 +314,82 @@ def softmax_anchor(q, k, v, grid, rope_split, heads, gate=None, scale=None,
         if rows is not None:
             g = g[:, rows]
         out = sigmoid(g) * out
+    return out
+
+
+# --------------------------------------------------------------------------
+# block-sparse softmax anchor (reading of [SV2] Experiments / [SV2-abs]:
+# the deployment stack applies sparse attention to the softmax anchors; the
+# pages give no pattern)
+# --------------------------------------------------------------------------
+
+Q_BLOCK = 256   # query rows per block (reading)
+K_TILE = 128    # keys per tile (reading)
+
+
+def anchor_block_scores(q, k, grid, rope_split, heads, scale=None, t_offset=0):
+    """Pooled-logit score of every (query block, key tile) pair.
+
+    Reading: q_bar = mean over the block's tokens of RoPE(Q) * scale, k_bar =
+    mean over the tile's tokens of RoPE(K); score = q_bar . k_bar (the mean
+    logit of the block pair).  Returns [B, heads, n_qblocks, n_ktiles]."""
+    qh = _heads(np.asarray(q, np.float64), heads)
+    kh = _heads(np.asarray(k, np.float64), heads)
+    D = qh.shape[-1]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    ang = rope_angles(*grid, *rope_split, t_offset=t_offset)
+    qh = apply_rope(qh, ang) * scale
+    kh = apply_rope(kh, ang)
+    N = qh.shape[2]
+    nqb = -(-N // Q_BLOCK)
+    nkt = -(-N // K_TILE)
+    qbar = np.stack([qh[:, :, i * Q_BLOCK:(i + 1) * Q_BLOCK].mean(axis=2) for i in range(nqb)], axis=2)
+    kbar = np.stack([kh[:, :, t * K_TILE:(t + 1) * K_TILE].mean(axis=2) for t in range(nkt)], axis=2)
+    return qbar @ np.swapaxes(kbar, -1, -2)
+
+
+def anchor_block_select(scores, keep):
+    """Top-`keep` key tiles of every query block by score, ties to the lower
+    tile index, returned in ascending tile order: int array [..., keep]."""
+    scores = np.asarray(scores, np.float64)
+    lead = scores.shape[:-1]
+    n = scores.shape[-1]
+    flat = scores.reshape(-1, n)
+    out = np.empty((flat.shape[0], keep), np.int64)
+    for r in range(flat.shape[0]):
+        order = sorted(range(n), key=lambda t: (-flat[r, t], t))
+        out[r] = sorted(order[:keep])
+    return out.reshape(*lead, keep)
+
+
+def softmax_anchor_tiles(q, k, v, grid, rope_split, heads, tiles, gate=None, scale=None,
+                         rows=None, t_offset=0):
+    """The gated softmax anchor with each query restricted to the keys of the
+    tiles kept for its block: tiles [B, heads, n_qblocks, keep] (distinct
+    indices of 128-key tiles).  Softmax over exactly those keys."""
+    qh = _heads(np.asarray(q, np.float64), heads)
+    kh = _heads(np.asarray(k, np.float64), heads)
+    vh = _heads(np.asarray(v, np.float64), heads)
+    B, nh, N, D = qh.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    ang = rope_angles(*grid, *rope_split, t_offset=t_offset)
+    qh = apply_rope(qh, ang)
+    kh = apply_rope(kh, ang)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.zeros((B, nh, len(rows), D))
+    key_tile = np.arange(N) // K_TILE
+    for b in range(B):
+        for h in range(nh):
+            for ri, i in enumerate(rows):
+                allowed = np.isin(key_tile, tiles[b, h, i // Q_BLOCK])
+                lg = (kh[b, h, allowed] @ qh[b, h, i]) * scale
+                p = np.exp(lg - lg.max())
+                out[b, h, ri] = (p / p.sum()) @ vh[b, h, allowed]
+    out = _merge(out)
+    if gate is not None:
+        out = sigmoid(np.asarray(gate, np.float64)[:, rows]) * out
     return out
 
 

@@ -357,6 +357,64 @@ def test_anchor_special_cases():
     assert rel(a, b) < 1e-12
 
 
+# ------------------------------------------- block-sparse anchor (reading)
+
+def _sparse_inputs(N, heads, D, seed_scale=1.0):
+    return (rand(1, N, heads * D) * seed_scale, rand(1, N, heads * D) * seed_scale,
+            rand(1, N, heads * D), rand(1, N, heads * D))
+
+
+def test_block_scores_are_mean_logits_of_each_block_pair():
+    """q_bar . k_bar = mean over the block pair of the full logit matrix
+    (bilinearity), including a ragged last block and tile (N = 600)."""
+    grid, split, heads, D = (2, 15, 20), (2, 1, 1), 2, 8
+    N = 600
+    q, k, _, _ = _sparse_inputs(N, heads, D)
+    sc = orc.anchor_block_scores(q, k, grid, split, heads)
+    ang = orc.rope_angles(*grid, *split)
+    for h in range(heads):
+        sl = slice(h * D, (h + 1) * D)
+        L = (orc.apply_rope(q[0, :, sl], ang) @ orc.apply_rope(k[0, :, sl], ang).T) * D ** -0.5
+        for qb in range(3):
+            for kt in range(5):
+                blk = L[qb * 256:(qb + 1) * 256, kt * 128:(kt + 1) * 128]
+                assert abs(sc[0, h, qb, kt] - blk.mean()) < 1e-12 * max(1.0, abs(blk).max())
+
+
+def test_block_selection_matches_a_stable_sort_and_breaks_ties_low():
+    scores = rand(3, 17)
+    scores[1, [2, 9, 11]] = scores[1].max() + 1.0  # a three-way tie at the top
+    sel = orc.anchor_block_select(scores, 5)
+    for r in range(3):
+        ref = np.sort(np.argsort(-scores[r], kind="stable")[:5])
+        assert np.array_equal(sel[r], ref)
+    assert {2, 9, 11} <= set(sel[1].tolist())
+    assert np.array_equal(orc.anchor_block_select(scores[1:2], 2), [[2, 9]])
+
+
+def test_tile_restricted_anchor_equals_dense_when_all_kept_and_gathered_softmax():
+    grid, split, heads, D = (2, 15, 20), (2, 1, 1), 2, 8
+    N = 600
+    q, k, v, g = _sparse_inputs(N, heads, D)
+    nkt = 5
+    all_tiles = np.broadcast_to(np.arange(nkt), (1, heads, 3, nkt))
+    dense = orc.softmax_anchor(q, k, v, grid, split, heads, gate=g)
+    assert rel(orc.softmax_anchor_tiles(q, k, v, grid, split, heads, all_tiles, gate=g), dense) < 1e-12
+    # two tiles per block, different per head and block: each row equals a
+    # plain softmax over the gathered keys (naive, no max subtraction)
+    tiles = np.array([[[[0, 4], [1, 2], [3, 4]], [[2, 3], [0, 1], [1, 4]]]])
+    rows = np.array([0, 255, 256, 511, 599])
+    y = orc.softmax_anchor_tiles(q, k, v, grid, split, heads, tiles, rows=rows)
+    ang = orc.rope_angles(*grid, *split)
+    for h in range(heads):
+        sl = slice(h * D, (h + 1) * D)
+        qr, kr = orc.apply_rope(q[0, :, sl], ang), orc.apply_rope(k[0, :, sl], ang)
+        for ri, i in enumerate(rows):
+            keys = np.concatenate([np.arange(t * 128, min((t + 1) * 128, N)) for t in tiles[0, h, i // 256]])
+            yn = orc.softmax_naive(qr[i:i + 1], kr[keys], v[0, keys, sl], D ** -0.5)
+            assert rel(y[0, ri:ri + 1, sl], yn) < 1e-12
+
+
 # ------------------------------------------------------------------ AttnRes (P6)
 
 def test_attnres_two_source_closed_form():
