@@ -356,7 +356,25 @@ def components(sana, args):
         ms = time_loop(f, 3)
         flops = 4 * WL.N * WL.N * WL.heads * WL.D
         out["softmax_anchor_720p"] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}
-        del q, k, v, g, y, ws
+        dense_ms = ms
+        # block-sparse anchor: each 256-query block keeps a quarter of the 591
+        # key tiles (selection by pooled logits included in the timing)
+        nkt = sana.anchor_tile_count(WL.N)
+        keep = (nkt + 3) // 4
+        ws = torch.empty(sana.softmax_anchor_sparse_workspace_size(1, (WL.T, WL.H, WL.W), WL.heads,
+                                                                   WL.D),
+                         dtype=torch.uint8, device="cuda")
+        tiles = torch.empty(1, WL.heads, (nkt + 1) // 2, keep, dtype=torch.int32, device="cuda")
+        f = lambda: sana.softmax_anchor_sparse_fwd(q, k, v, g, rope, (WL.T, WL.H, WL.W), WL.heads,
+                                                   keep, tiles=tiles, out=y, ws=ws)
+        f()
+        ms = time_loop(f, 5)
+        kept = 4 * WL.N * min(WL.N, keep * 128) * WL.heads * WL.D
+        out["softmax_anchor_sparse_720p_25pct"] = {
+            "ms": ms, "keep_tiles": keep, "key_tiles": nkt,
+            "TFLOP_per_s_executed": kept / (ms / 1e3) / 1e12,
+            "speedup_vs_dense": dense_ms / ms}
+        del q, k, v, g, y, ws, tiles
     except Exception as e:  # not built yet
         out["softmax_anchor_720p"] = {"unavailable": str(e)[:200]}
     # whole stacks on the 720p/5s grid: the 4-layer 3:1 group (no AttnRes, no

@@ -196,6 +196,37 @@ SANA_API sana_status sana_softmax_anchor_fwd(const sana_shape* shape, sana_dtype
                                     size_t ws_bytes, sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Block-sparse gated softmax anchor ([SV2] Experiments and [SV2a]: the
+ * deployment stack applies sparse attention to the softmax anchors; the
+ * pattern below is this library's reading, the pages give none).
+ * Queries form blocks of 256 tokens and keys tiles of 128 tokens; every query
+ * block attends to exactly the keys of the `keep_tiles` key tiles listed for
+ * it, with the softmax taken over those keys (same RoPE, scale and gate as
+ * sana_softmax_anchor_fwd).
+ * tiles: device int32 [B][heads][ceil(ceil(N/128)/2)][keep_tiles].
+ *   select_tiles != 0: the library fills it: per block, the keep_tiles key
+ *     tiles with the largest pooled logit mean(RoPE(Q)*scale) . mean(RoPE(K))
+ *     over the block's and the tile's tokens, ties to the lower index, listed
+ *     in ascending order.
+ *   select_tiles == 0: the caller's list is used as given; entries must be
+ *     distinct and in [0, ceil(N/128)) (other values give undefined results;
+ *     loads stay in bounds).
+ * 1 <= keep_tiles <= ceil(N/128); keep_tiles = ceil(N/128) is the dense
+ * anchor.  bf16 only (head_dim 128); N <= 2^21.  Workspace:
+ * sana_softmax_anchor_sparse_workspace_size() bytes (rotated Q, K and the
+ * per-tile sums of the selection).
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_softmax_anchor_sparse_workspace_size(const sana_shape* shape,
+                                                          sana_dtype dtype);
+SANA_API sana_status sana_softmax_anchor_sparse_fwd(const sana_shape* shape, sana_dtype dtype,
+                                                    const void* q, const void* k, const void* v,
+                                                    const void* gate_logits,
+                                                    const sana_rope* rope, float scale,
+                                                    int keep_tiles, int* tiles, int select_tiles,
+                                                    void* out, void* ws, size_t ws_bytes,
+                                                    sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Block Attention Residuals router ([SV2] AttnRes equation, timestep term 0):
  *   l_i = w . v_i / sqrt(mean_c v_i^2 + rms_eps),  alpha = softmax_i(l),
  *   h = sum_i alpha_i v_i,   per token, over num_sources sources.

@@ -89,6 +89,11 @@ def _load():
         "sana_softmax_anchor_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, POINTER(RopeStruct), c_float, c_void_p,
                                             c_void_p, c_size_t, c_void_p]),
+        "sana_softmax_anchor_sparse_workspace_size": (c_size_t, [POINTER(Shape), c_int]),
+        "sana_softmax_anchor_sparse_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p,
+                                                   c_void_p, c_void_p, POINTER(RopeStruct),
+                                                   c_float, c_int, c_void_p, c_int, c_void_p,
+                                                   c_void_p, c_size_t, c_void_p]),
         "sana_attnres_route": (c_int, [c_int, c_longlong, c_int, c_int, POINTER(c_void_p), c_int,
                                        c_void_p, c_float, c_void_p, c_void_p, c_void_p]),
         "sana_gemm_bf16": (c_int, [c_longlong, c_int, c_int, c_void_p, c_longlong, c_void_p,
@@ -309,6 +314,43 @@ def softmax_anchor_fwd(q, k, v, gate, rope, grid, heads, scale=0.0, out=None, ws
         None if rope is None else ctypes.byref(rope.struct), scale, _ptr(out), _ptr(ws), ws.numel(),
         _stream()))
     return out
+
+
+def anchor_tile_count(N: int) -> int:
+    """Key tiles of 128 tokens; query blocks are pairs of them."""
+    return (N + 127) // 128
+
+
+def softmax_anchor_sparse_workspace_size(B, grid, heads, head_dim) -> int:
+    s = make_shape(B, grid, heads, head_dim)
+    return lib.sana_softmax_anchor_sparse_workspace_size(ctypes.byref(s), SANA_BF16)
+
+
+def softmax_anchor_sparse_fwd(q, k, v, gate, rope, grid, heads, keep_tiles, tiles=None,
+                              select=True, scale=0.0, out=None, ws=None):
+    """Block-sparse gated softmax anchor (bf16).  With select, the library picks
+    the keep_tiles key tiles of every 256-query block and writes them into
+    `tiles` (allocated if None); without, the given int32 tiles
+    [B, heads, n_blocks, keep_tiles] are used.  Returns (out, tiles)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    B, N, C = q.shape
+    D = C // heads
+    dt = _dtype_code(q)
+    s = make_shape(B, grid, heads, D)
+    nt = anchor_tile_count(N)
+    if tiles is None:
+        tiles = torch.empty(B, heads, (nt + 1) // 2, keep_tiles, dtype=torch.int32, device=q.device)
+    _need(tiles, "tiles")
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = _ws(lib.sana_softmax_anchor_sparse_workspace_size(ctypes.byref(s), dt), q.device)
+    check(lib.sana_softmax_anchor_sparse_fwd(
+        ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate),
+        None if rope is None else ctypes.byref(rope.struct), scale, keep_tiles, _ptr(tiles),
+        int(bool(select)), _ptr(out), _ptr(ws), ws.numel(), _stream()))
+    return out, tiles
 
 
 # ---------------------------------------------------------------- AttnRes, norm, GEMM

@@ -19,6 +19,10 @@
 //                   and TMA store.
 // TMEM (512 columns): S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512);
 // P_i occupies the first 64 columns of S_i.
+//
+// Block-sparse form: with a tile list, the CTA walks only the `keep` key tiles
+// listed for its 256-query block (in list order) instead of all of them; the
+// softmax is exact over the keys of those tiles.
 #include <cuda.h>
 
 #include "sana_common.cuh"
@@ -123,11 +127,12 @@ struct AnchorCtl {
 
 // 320 threads = 10 warps: three share one of the four 16K-register slices of
 // the SM, which caps a thread at 168 registers.
-template <bool kGate>
+template <bool kGate, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     anchor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                  const __grid_constant__ CUtensorMap tm_y, int N, int* status) {
+                  const __grid_constant__ CUtensorMap tm_y, int N, const int* __restrict__ tiles,
+                  int keep, int* status) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ AnchorCtl ctl;
   uint8_t* smem = align1024(smem_raw);
@@ -140,6 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int row0 = qp * 2 * kRows;  // first query row of tile 0
   const int nkv = (N + kRows - 1) / kRows;
   const int kv_tail = N - (nkv - 1) * kRows;  // valid keys in the last tile
+  // key tiles this CTA visits: all of them, or the `keep` listed for its block
+  const int* list = kSparse ? tiles + ((size_t)(b * gridDim.y + h) * gridDim.x + qp) * keep : nullptr;
+  const int nk_all = kSparse ? keep : nkv;
+  auto key_tile = [&](int j) { return kSparse ? __ldg(list + j) : j; };
   const WaitCtx wc{&ctl.abort_flag, status};
 
   if (tid == 0) {
@@ -184,28 +193,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int nk = 0, nv = 0;
       bool ok = true;
-      for (int j = 0; j < nkv; ++j) {
+      for (int j = 0; j < nk_all; ++j) {
         const int sk = j % kKS, sv = j % kVS;
+        const int row = key_tile(j) * kRows;  // first key of the tile
         if (j >= kKS && !mbar_wait(&ctl.k_empty[sk], ((j / kKS) - 1) & 1, wc, 0x31)) {
           ok = false;
           break;
         }
         mbar_arrive_expect_tx(&ctl.k_full[sk], kTileB);
-        tma_load_3d(k_s + sk * kTileB, &tm_k, &ctl.k_full[sk], h * kD, j * kRows, b);
-        tma_load_3d(k_s + sk * kTileB + kHalf, &tm_k, &ctl.k_full[sk], h * kD + 64, j * kRows, b);
+        tma_load_3d(k_s + sk * kTileB, &tm_k, &ctl.k_full[sk], h * kD, row, b);
+        tma_load_3d(k_s + sk * kTileB + kHalf, &tm_k, &ctl.k_full[sk], h * kD + 64, row, b);
         ++nk;
         if (j >= kVS && !mbar_wait(&ctl.v_empty[sv], ((j / kVS) - 1) & 1, wc, 0x32)) {
           ok = false;
           break;
         }
         mbar_arrive_expect_tx(&ctl.v_full[sv], kTileB);
-        tma_load_3d(v_s + sv * kTileB, &tm_v, &ctl.v_full[sv], h * kD, j * kRows, b);
-        tma_load_3d(v_s + sv * kTileB + kHalf, &tm_v, &ctl.v_full[sv], h * kD + 64, j * kRows, b);
+        tma_load_3d(v_s + sv * kTileB, &tm_v, &ctl.v_full[sv], h * kD, row, b);
+        tma_load_3d(v_s + sv * kTileB + kHalf, &tm_v, &ctl.v_full[sv], h * kD + 64, row, b);
         ++nv;
       }
       // G goes into the K ring once the last S MMAs have read it
       if (ok && kGate) {
-        for (int j = (nkv > kKS ? nkv - kKS : 0); j < nkv && ok; ++j)
+        for (int j = (nk_all > kKS ? nk_all - kKS : 0); j < nk_all && ok; ++j)
           ok = mbar_wait(&ctl.k_empty[j % kKS], (j / kKS) & 1, wc, 0x3c);
         if (ok) {
           mbar_arrive_expect_tx(&ctl.g_full, 2 * kTileB);
@@ -253,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   idesc_o, (j | kk) != 0);
         umma_commit(&ctl.pv_done[i]);
       };
-      bool ok = mbar_wait(&ctl.q_full, 0, wc, 0x33) && nkv > 0 &&
+      bool ok = mbar_wait(&ctl.q_full, 0, wc, 0x33) && nk_all > 0 &&
                 mbar_wait(&ctl.k_full[0], 0, wc, 0x36);
       if (ok) {
         tc_fence_after();
@@ -261,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(1, 0);
         umma_commit(&ctl.k_empty[0]);  // K'_0 is read by these two only
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const bool more = j + 1 < nkv;
+      for (int j = 0; ok && j < nk_all; ++j) {
+        const bool more = j + 1 < nk_all;
         if (!mbar_wait(&ctl.v_full[j % kVS], (j / kVS) & 1, wc, 0x35)) break;
         if (more && !mbar_wait(&ctl.k_full[(j + 1) % kKS], ((j + 1) / kKS) & 1, wc, 0x36)) break;
         for (int i = 0; i < 2 && ok; ++i) {
@@ -296,14 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_s = tmem + qi * 128, tmem_o = tmem + 256 + qi * 128;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; ok && j < nkv; ++j) {
+    for (int j = 0; ok && j < nk_all; ++j) {
       // warp-uniform outcome: tcgen05.ld / st are warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(&ctl.s_full[qi], j & 1, wc, 0x38))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const bool last = j == nkv - 1 && kv_tail < kRows;
+      const bool last = key_tile(j) == nkv - 1 && kv_tail < kRows;
       // pass 1: row max, 64 columns in registers at a time (four independent
       // chains of 3-input max)
       float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -408,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------- epilogue: Y = O / l * sigmoid(G)
     ok = __all_sync(0xffffffffu,
-                    ok && nkv > 0 && mbar_wait(&ctl.pv_done[qi], (nkv - 1) & 1, wc, 0x3a));
+                    ok && nk_all > 0 && mbar_wait(&ctl.pv_done[qi], (nk_all - 1) & 1, wc, 0x3a));
     if (kGate) ok = ok && __all_sync(0xffffffffu, mbar_wait(&ctl.g_full, 0, wc, 0x3d));
     uint8_t* ybuf = q_s + qi * kTileB;  // Q'_i is no longer read
     const uint8_t* gbuf = k_s + qi * kTileB;
@@ -459,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kWarpMma) {
     if (*wc.abort_flag) {  // MMAs in flight finish before TMEM is freed
-      mbar_drain(&ctl.pv_done[0], (nkv - 1) & 1);
-      mbar_drain(&ctl.pv_done[1], (nkv - 1) & 1);
+      mbar_drain(&ctl.pv_done[0], (nk_all - 1) & 1);
+      mbar_drain(&ctl.pv_done[1], (nk_all - 1) & 1);
     }
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -472,7 +482,8 @@ constexpr size_t kAnchorSmem = 1024 + 2 * kTileB + kKS * kTileB + kVS * kTileB;
 }  // namespace
 
 sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr, const void* v,
-                            const void* gt, const GridDev& g, void* out, cudaStream_t st) {
+                            const void* gt, const GridDev& g, const int* tiles, int keep,
+                            void* out, cudaStream_t st) {
   const uint64_t C = (uint64_t)s.heads * kD, N = (uint64_t)g.N;
   CUtensorMap tq, tk, tv, tg, ty;
   bool okm = make_tmap_bf16_3d(&tq, qr, C, N, s.B, C, N * C, kRows) &&
@@ -486,18 +497,24 @@ sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr,
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr[dev]) {
-    cudaFuncSetAttribute(anchor_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kAnchorSmem);
-    cudaFuncSetAttribute(anchor_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kAnchorSmem);
+    const int bytes = (int)kAnchorSmem;
+    cudaFuncSetAttribute(anchor_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaFuncSetAttribute(anchor_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaFuncSetAttribute(anchor_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaFuncSetAttribute(anchor_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     attr[dev] = true;
   }
   const int qtiles = (g.N + kRows - 1) / kRows;
   const dim3 grid((qtiles + 1) / 2, s.heads, s.B);
-  if (gt)
-    anchor_kernel<true><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, status_word());
+  int* sw = status_word();
+  if (gt && tiles)
+    anchor_kernel<true, true><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, tiles, keep, sw);
+  else if (gt)
+    anchor_kernel<true, false><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, nullptr, 0, sw);
+  else if (tiles)
+    anchor_kernel<false, true><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, tiles, keep, sw);
   else
-    anchor_kernel<false><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, status_word());
+    anchor_kernel<false, false><<<grid, kThreads, kAnchorSmem, st>>>(tq, tk, tv, tg, ty, g.N, nullptr, 0, sw);
   return check_launch("anchor_kernel");
 }
 

@@ -298,8 +298,6 @@ sana_status rope_rotate_run(const void* x, bool bf16, const RopeDev* rope, const
 sana_status anchor_f32_run(const sana_shape& s, const float* qr, const float* kr, const float* v,
                            const float* gt, const GridDev& g, float scale, float* out,
                            cudaStream_t st);
-sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr, const void* v,
-                            const void* gt, const GridDev& g, void* out, cudaStream_t st);
 
 size_t anchor_ws_bytes(const sana_shape& s, sana_dtype dt) {
   const size_t n = (size_t)s.B * s.T * s.H * s.W * s.heads * s.head_dim;
@@ -328,13 +326,51 @@ sana_status anchor_run(const sana_shape& s, sana_dtype dt, const void* q, const 
     const float qmul = scale * 1.4426950408889634f;
     if (sana_status e = rope_rotate_run(q, true, rope, g, s.B, D, qmul, qr, st)) return e;
     if (sana_status e = rope_rotate_run(k, true, rope, g, s.B, D, 1.f, kr, st)) return e;
-    return anchor_bf16_run(s, qr, kr, v, gt, g, out, st);
+    return anchor_bf16_run(s, qr, kr, v, gt, g, nullptr, 0, out, st);
   }
   if (sana_status e = rope_rotate_run(q, false, rope, g, s.B, D, 1.f, qr, st)) return e;
   if (sana_status e = rope_rotate_run(k, false, rope, g, s.B, D, 1.f, kr, st)) return e;
   return anchor_f32_run(s, static_cast<const float*>(qr), static_cast<const float*>(kr),
                         static_cast<const float*>(v), static_cast<const float*>(gt), g, scale,
                         static_cast<float*>(out), st);
+}
+
+// Sparse form (bf16): the same prepass, then (if select) the tile selection,
+// then the anchor kernel over the listed tiles.
+size_t anchor_sparse_ws_bytes(const sana_shape& s) {
+  const size_t N = (size_t)s.T * s.H * s.W;
+  const size_t ntiles = (N + 127) / 128;
+  Carver cv(nullptr, ~size_t(0));
+  cv.take<char>(anchor_ws_bytes(s, SANA_BF16));
+  cv.take<float>((size_t)s.B * ntiles * s.heads * s.head_dim);
+  cv.take<float>((size_t)s.B * ntiles * s.heads * s.head_dim);
+  return align_up(cv.used, 256);
+}
+
+sana_status anchor_sparse_run(const sana_shape& s, const void* q, const void* k, const void* v,
+                              const void* gt, const RopeDev* rope, float scale, int keep, int* tiles,
+                              bool select, void* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const GridDev g = to_grid(s);
+  if (g.N == 0) return SANA_OK;
+  const size_t need = anchor_sparse_ws_bytes(s);
+  if (ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "sparse anchor: workspace %zu < %zu bytes", ws_bytes, need);
+  const size_t n = (size_t)s.B * g.N * s.heads * s.head_dim;
+  const size_t ntiles = ((size_t)g.N + 127) / 128;
+  Carver cv(ws, ws_bytes);
+  void* qr = cv.take<char>(n * 2);
+  void* kr = cv.take<char>(n * 2);
+  cv.used = align_up(anchor_ws_bytes(s, SANA_BF16), 256);
+  float* qsums = cv.take<float>((size_t)s.B * ntiles * s.heads * s.head_dim);
+  float* ksums = cv.take<float>((size_t)s.B * ntiles * s.heads * s.head_dim);
+  if (scale <= 0.f) scale = 1.f / sqrtf((float)s.head_dim);
+  const float qmul = scale * 1.4426950408889634f;
+  if (sana_status e = rope_rotate_run(q, true, rope, g, s.B, s.head_dim, qmul, qr, st)) return e;
+  if (sana_status e = rope_rotate_run(k, true, rope, g, s.B, s.head_dim, 1.f, kr, st)) return e;
+  if (select)
+    if (sana_status e = anchor_select_run(s.B, g.N, s.heads, qr, kr, keep, qsums, ksums, tiles, st))
+      return e;
+  return anchor_bf16_run(s, qr, kr, v, gt, g, tiles, keep, out, st);
 }
 
 }  // namespace sana
@@ -575,6 +611,56 @@ sana_status sana_softmax_anchor_fwd(const sana_shape* s, sana_dtype dt, const vo
   RopeDev rd{};
   if (rope) rd = to_dev(*rope);
   return anchor_run(*s, dt, q, k, v, g, rope ? &rd : nullptr, scale, out, ws, ws_bytes, stream);
+}
+
+size_t sana_softmax_anchor_sparse_workspace_size(const sana_shape* s, sana_dtype dt) {
+  if (check_shape(s, dt, "sana_softmax_anchor_sparse_workspace_size") != SANA_OK ||
+      dt != SANA_BF16)
+    return 0;
+  return anchor_sparse_ws_bytes(*s);
+}
+
+sana_status sana_softmax_anchor_sparse_fwd(const sana_shape* s, sana_dtype dt, const void* q,
+                                           const void* k, const void* v, const void* g,
+                                           const sana_rope* rope, float scale, int keep_tiles,
+                                           int* tiles, int select_tiles, void* out, void* ws,
+                                           size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_softmax_anchor_sparse_fwd";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (dt != SANA_BF16) return fail(SANA_ERR_UNSUPPORTED, "%s: bf16 only", who);
+  if (rope)
+    if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!std::isfinite(scale)) return fail(SANA_ERR_INVALID_ARG, "%s: scale is not finite", who);
+  if (s->T == 0) return SANA_OK;
+  const long long N = (long long)s->T * s->H * s->W;
+  const long long ntiles = (N + 127) / 128;
+  if (ntiles > kAnchorMaxTiles)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: %lld key tiles (max %d)", who, ntiles, kAnchorMaxTiles);
+  if (keep_tiles < 1 || keep_tiles > ntiles)
+    return fail(SANA_ERR_INVALID_ARG, "%s: keep_tiles=%d outside [1, %lld]", who, keep_tiles, ntiles);
+  if (!q || !k || !v || !out || !tiles)
+    return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  const void* ptrs[6] = {q, k, v, g, out, tiles};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * N * s->heads * s->head_dim * 2;
+  const size_t tb = (size_t)s->B * s->heads * ((ntiles + 1) / 2) * keep_tiles * 4;
+  if (overlap(out, n, q, n) || overlap(out, n, k, n) || overlap(out, n, v, n) || overlap(out, n, g, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an input", who);
+  if (overlap(tiles, tb, out, n) || overlap(tiles, tb, q, n) || overlap(tiles, tb, k, n) ||
+      overlap(tiles, tb, v, n) || overlap(tiles, tb, g, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: tiles alias a tensor", who);
+  const size_t need = anchor_sparse_ws_bytes(*s);
+  if (!ws || ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  if (overlap(ws, need, tiles, tb) || overlap(ws, need, out, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace aliases the output or the tiles", who);
+  RopeDev rd{};
+  if (rope) rd = to_dev(*rope);
+  return anchor_sparse_run(*s, q, k, v, g, rope ? &rd : nullptr, scale, keep_tiles, tiles,
+                           select_tiles != 0, out, ws, ws_bytes, stream);
 }
 
 sana_status sana_attnres_route(int B, long long N, int C, sana_dtype dt, const void* const* sources,

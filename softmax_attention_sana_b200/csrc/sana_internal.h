@@ -140,6 +140,20 @@ sana_status anchor_run(const sana_shape& s, sana_dtype dt, const void* q, const 
                        const void* v, const void* g, const RopeDev* rope, float scale,
                        void* out, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// Block-sparse anchor: tile selection (anchor_select.cu) and the anchor kernel
+// over listed key tiles (anchor_tc.cu; tiles == nullptr visits every tile).
+constexpr int kAnchorMaxTiles = 16384;  // key tiles the selection supports (N <= 2M)
+size_t anchor_select_smem(int ntiles);
+sana_status anchor_select_run(int B, int N, int heads, const void* qr, const void* kr, int keep,
+                              float* qsums, float* ksums, int* tiles, cudaStream_t st);
+sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr, const void* v,
+                            const void* gt, const GridDev& g, const int* tiles, int keep,
+                            void* out, cudaStream_t st);
+size_t anchor_sparse_ws_bytes(const sana_shape& s);
+sana_status anchor_sparse_run(const sana_shape& s, const void* q, const void* k, const void* v,
+                              const void* g, const RopeDev* rope, float scale, int keep, int* tiles,
+                              bool select, void* out, void* ws, size_t ws_bytes, cudaStream_t st);
+
 // ---------------------------------------------------------------- AttnRes / norm / GEMM
 sana_status attnres_run(int B, long long N, int C, sana_dtype dt, const void* const* sources,
                         int S, const float* w, float eps, void* h, float* alpha, bool normed_out,

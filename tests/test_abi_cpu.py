@@ -138,6 +138,28 @@ def test_block_causal_scan_sizes_and_validation():
     assert _call_scan(s, 3, out=2 << 20) == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
 
 
+def test_sparse_anchor_sizes_and_validation():
+    L = _lib
+    s720 = _shape(T=21, H=45, W=80, heads=24, head_dim=128)
+    ws = L.lib.sana_softmax_anchor_sparse_workspace_size(ctypes.byref(s720), L.SANA_BF16)
+    # rotated Q and K (2 x 464.5 MB) + per-tile fp32 sums of both (2 x 591 x 3072 x 4 B)
+    assert ws >= 2 * 75600 * 3072 * 2 + 2 * 591 * 3072 * 4
+    assert L.lib.sana_softmax_anchor_sparse_workspace_size(ctypes.byref(_shape()), L.SANA_F32) == 0
+    r = _lib.RopeStruct(16, 16, 16, 16, 16, 16, 22, 21, 21, 2, 4, 4)
+    s = _shape(head_dim=128)  # N = 32: one key tile
+
+    def call(dtype=L.SANA_BF16, keep=1, tiles=6 << 20, ws_bytes=1 << 24):
+        return L.lib.sana_softmax_anchor_sparse_fwd(
+            ctypes.byref(s), dtype, 1 << 20, 2 << 20, 3 << 20, None, ctypes.byref(r), 0.0, keep,
+            tiles, 1, 4 << 20, 1 << 26, ws_bytes, None)
+    assert call(dtype=L.SANA_F32) == L.SANA_ERR_UNSUPPORTED
+    assert call(keep=0) == L.SANA_ERR_INVALID_ARG and "keep_tiles" in L.last_error()
+    assert call(keep=2) == L.SANA_ERR_INVALID_ARG
+    assert call(tiles=None) == L.SANA_ERR_INVALID_ARG
+    assert call(tiles=4 << 20) == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
+    assert call(ws_bytes=64) == L.SANA_ERR_WORKSPACE
+
+
 def test_attnres_and_gemm_validation():
     L = _lib
     arr = (ctypes.c_void_p * 1)(4096)
