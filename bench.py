@@ -515,6 +515,57 @@ def run_anchor_only(args):
     print(json.dumps({"anchor_480p_ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}), flush=True)
 
 
+def run_scan_only(args):
+    """The whole 720p/60s sequence through the block-causal scan (81 blocks,
+    867,600 tokens, inputs drawn on the device): K steps, ms per call."""
+    import softmax_attention_sana_b200 as sana
+    wl = si.LONG
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4000)
+    q, k, v = (torch.randn((1, wl.N, wl.C), generator=gen, device="cuda", dtype=torch.bfloat16)
+               for _ in range(3))
+    rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
+    S = torch.zeros(1, wl.heads, wl.D, wl.D, device="cuda")
+    z = torch.zeros(1, wl.heads, wl.D, device="cuda")
+    ws = torch.empty(sana.linattn_block_causal_scan_workspace_size(1, (wl.T, wl.H, wl.W), wl.heads,
+                                                                   wl.D, 3, 1),
+                     dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(q)
+    f = lambda: sana.linattn_block_causal_scan(q, k, v, None, rope, (wl.T, wl.H, wl.W), 0,
+                                               wl.heads, 3, S, z, commit=False, out=y, ws=ws)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    nb = 4 * wl.N * wl.C * 2 + 2 * wl.heads * (wl.D * wl.D + wl.D) * 4
+    print(json.dumps({"scan_720p60s_ms": ms, "tokens_per_s": wl.N / (ms / 1e3),
+                      "GB_per_s": nb / (ms / 1e3) / 1e9}), flush=True)
+
+
+def run_sparse_only(args):
+    """The block-sparse anchor on the 720p/5s grid, a quarter of the key tiles
+    per 256-query block (selection included): K steps, ms per call."""
+    import softmax_attention_sana_b200 as sana
+    q, k, v, g = (t.cuda() for t in si.qkvg(WL))
+    grid = (WL.T, WL.H, WL.W)
+    rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
+    nkt = sana.anchor_tile_count(WL.N)
+    keep = (nkt + 3) // 4
+    y = torch.empty_like(q)
+    ws = torch.empty(sana.softmax_anchor_sparse_workspace_size(1, grid, WL.heads, WL.D),
+                     dtype=torch.uint8, device="cuda")
+    tiles = torch.empty(1, WL.heads, (nkt + 1) // 2, keep, dtype=torch.int32, device="cuda")
+    f = lambda: sana.softmax_anchor_sparse_fwd(q, k, v, g, rope, grid, WL.heads, keep, tiles=tiles,
+                                               out=y, ws=ws)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    kept = 4 * WL.N * min(WL.N, keep * 128) * WL.heads * WL.D
+    print(json.dumps({"sparse_anchor_720p_25pct_ms": ms, "keep_tiles": keep,
+                      "TFLOP_per_s_executed": kept / (ms / 1e3) / 1e12}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -533,6 +584,10 @@ def main():
                     help="also time the 4-layer group and the 16-layer AttnRes stack")
     ap.add_argument("--anchor-only", action="store_true",
                     help="run only the 480p-shaped softmax anchor (a small case for profiling)")
+    ap.add_argument("--scan-only", action="store_true",
+                    help="run only the whole-sequence block-causal scan at 720p/60s")
+    ap.add_argument("--sparse-only", action="store_true",
+                    help="run only the block-sparse anchor at 720p/5s (25%% of the key tiles)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -541,6 +596,12 @@ def main():
     try:
         if args.anchor_only:
             run_anchor_only(args)
+            return
+        if args.scan_only:
+            run_scan_only(args)
+            return
+        if args.sparse_only:
+            run_sparse_only(args)
             return
         if args.impl == "reference":
             run_reference(args, world, rank)
