@@ -163,6 +163,50 @@ __global__ void rope_rotate_kernel(const T* __restrict__ x, RopeDev rope, GridDe
   }
 }
 
+// bf16 form: one 16-byte chunk (4 rotary pairs of one head) per thread and
+// iteration, so loads and stores are full-width; the token's grid position is
+// decoded once per chunk.
+__global__ void __launch_bounds__(256)
+    rope_rotate_bf16x8_kernel(const uint4* __restrict__ x, RopeDev rope, GridDev g, int D,
+                              float mul, uint4* __restrict__ out) {
+  const int b = blockIdx.y;
+  const int chunks = g.heads * D / 8;  // per token
+  const long long total = (long long)g.N * chunks;
+  const int hw = g.H * g.W;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / chunks);
+    const int c = (int)(i - (long long)n * chunks);
+    const int j0 = (c * 8 % D) / 2;  // first rotary pair of the chunk within its head
+    const size_t off = (size_t)b * total + i;
+    const uint4 raw = x[off];
+    uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    const int t = n / hw, rem = n - t * hw, hh = rem / g.W, ww = rem - hh * g.W;
+    const int tt = g.t_offset + b * g.t_stride + t;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 v = bf2_to_f2(w[k]);
+      if (rope.cos_t) {
+        const int j = j0 + k;
+        float cs, sn;
+        if (j < rope.n_t) {
+          cs = rope.cos_t[tt * rope.n_t + j];
+          sn = rope.sin_t[tt * rope.n_t + j];
+        } else if (j < rope.n_t + rope.n_h) {
+          cs = rope.cos_h[hh * rope.n_h + (j - rope.n_t)];
+          sn = rope.sin_h[hh * rope.n_h + (j - rope.n_t)];
+        } else {
+          cs = rope.cos_w[ww * rope.n_w + (j - rope.n_t - rope.n_h)];
+          sn = rope.sin_w[ww * rope.n_w + (j - rope.n_t - rope.n_h)];
+        }
+        v = rotate(v.x, v.y, make_float2(cs, sn));
+      }
+      w[k] = f2_to_bf2(v.x * mul, v.y * mul);
+    }
+    out[off] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // One thread per (query, head, batch): online softmax over all keys in fp32.
 template <int D>
 __global__ void __launch_bounds__(128)
@@ -310,7 +354,13 @@ sana_status rope_rotate_run(const void* x, bool bf16, const RopeDev* rope, const
   int blocks = (int)((pairs + 255) / 256);
   if (blocks > 4 * kNumSMs * 8) blocks = 4 * kNumSMs * 8;
   if (blocks < 1) blocks = 1;
-  if (bf16)
+  if (bf16 && D % 8 == 0) {
+    const long long chunks = (long long)g.N * g.heads * D / 8;
+    long long cb = (chunks + 255) / 256;
+    if (cb > 8 * kNumSMs * 8) cb = 8 * kNumSMs * 8;
+    rope_rotate_bf16x8_kernel<<<dim3((unsigned)(cb > 0 ? cb : 1), B), 256, 0, st>>>(
+        static_cast<const uint4*>(x), r, g, D, mul, static_cast<uint4*>(out));
+  } else if (bf16)
     rope_rotate_kernel<__nv_bfloat16><<<dim3(blocks, B), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), r, g, D, mul, static_cast<__nv_bfloat16*>(out));
   else
