@@ -45,6 +45,10 @@ Readings where the pages are silent (each also listed in the design doc):
   left out while it is empty.
 * Stack: layer l is an anchor iff l % 4 == 3; FFN = W_down SiLU(W_up x) with
   hidden size ffn_mult * C; sublayer input RMSNorm(h) without gain.
+* Backward: the pages train from scratch ([SV1] sec. 4 training setup) but
+  print no backward; linattn_backward is the chain rule through the forward
+  as written (ReLU derivative 1 for x > 0, 0 otherwise), pinned by finite
+  differences.
 * Sparse anchor ([SV2] Experiments and [SV2-abs] say only that the
   deployment stack applies sparse attention to the softmax anchors): queries
   in blocks of 256 tokens, keys in tiles of 128; each block keeps the `keep`
@@ -174,6 +178,54 @@ def linattn_bidirectional(q, k, v, grid, rope_split, heads, gate=None, eps=EPS,
     S, z = linattn_state(k, v, ang, heads)
     y = linattn_apply(q, S, z, ang, heads, gate, eps)
     return y, S, z
+
+
+def rope_transpose(x, angles):
+    """Inverse (= transpose) of apply_rope: rotate pairs by -angle."""
+    return apply_rope(x, -angles)
+
+
+def linattn_backward(q, k, v, grid, rope_split, heads, dy, gate=None, eps=EPS, t_offset=0):
+    """Gradients of linattn_bidirectional's Y with respect to Q, K, V and G.
+
+    The forward ([SV1] sec. 3.2, gated per [SV2-abs]) differentiated step by
+    step in reverse; the pages train the model from scratch but print no
+    backward, so this is the chain rule applied to the forward as written:
+      o_i = num_i / den_i, num_i = q'_i S, den_i = phi(q_i) . z + eps,
+      y_i = sigmoid(g_i) * o_i.
+    Returns (dQ, dK, dV, dG) with dG None when there is no gate."""
+    T, H, W = grid
+    ang = rope_angles(T, H, W, *rope_split, t_offset=t_offset)
+    qh = _heads(np.asarray(q, np.float64), heads)
+    kh = _heads(np.asarray(k, np.float64), heads)
+    vh = _heads(np.asarray(v, np.float64), heads)
+    dyh = _heads(np.asarray(dy, np.float64), heads)
+    q_phi, k_phi = phi(qh), phi(kh)
+    q_rope, k_rope = apply_rope(q_phi, ang), apply_rope(k_phi, ang)
+    S = np.swapaxes(k_rope, -1, -2) @ vh
+    z = k_phi.sum(axis=2)
+    num = q_rope @ S
+    den = (q_phi @ z[..., :, None])[..., 0] + eps
+    o = num / den[..., None]
+    if gate is not None:
+        sg = sigmoid(_heads(np.asarray(gate, np.float64), heads))
+        dg = dyh * o * sg * (1.0 - sg)
+        do = dyh * sg
+    else:
+        dg = None
+        do = dyh
+    dnum = do / den[..., None]                        # d/d num_i
+    dden = -(do * o).sum(axis=-1) / den               # d/d den_i
+    dq_rope = dnum @ np.swapaxes(S, -1, -2)           # d/d q'_i = dnum_i S^T
+    dS = np.swapaxes(q_rope, -1, -2) @ dnum           # sum_i q'_i^T dnum_i
+    dz = (dden[..., None] * q_phi).sum(axis=2)        # sum_i dden_i phi(q_i)
+    dq_phi = rope_transpose(dq_rope, ang) + dden[..., None] * z[..., None, :]
+    dk_rope = vh @ np.swapaxes(dS, -1, -2)            # d/d k'_j = v_j dS^T
+    dv = k_rope @ dS                                  # d/d v_j = k'_j dS
+    dk_phi = rope_transpose(dk_rope, ang) + dz[..., None, :]
+    dq = dq_phi * (qh > 0)
+    dk = dk_phi * (kh > 0)
+    return _merge(dq), _merge(dk), _merge(dv), None if dg is None else _merge(dg)
 
 
 def linattn_bruteforce(q, k, v, grid, rope_split, heads, gate=None, eps=EPS,

@@ -251,6 +251,56 @@ def test_block_sequence_resumes_from_a_carried_state():
     assert rel(y_n, y_r) == 0 and np.array_equal(S_n, S_a) and np.array_equal(z_n, z_a)
 
 
+@pytest.mark.parametrize("gated,B,grid,split,heads,D", [
+    (True, 1, (2, 3, 4), (2, 1, 1), 2, 8),
+    (False, 2, (3, 5, 7), (2, 3, 3), 1, 16),   # N = 105
+    (True, 2, (1, 1, 1), (0, 0, 4), 2, 8),     # a single token
+])
+def test_backward_matches_central_finite_differences(gated, B, grid, split, heads, D):
+    """<dL/dx, u> for L = sum(dY * Y) against (L(x + h u) - L(x - h u)) / 2h,
+    for a random direction u in each of Q, K, V (and G)."""
+    N = grid[0] * grid[1] * grid[2]
+    C = heads * D
+    q, k, v, dy = (rand(B, N, C) for _ in range(4))
+    g = rand(B, N, C) if gated else None
+    grads = orc.linattn_backward(q, k, v, grid, split, heads, dy, gate=g)
+
+    def loss(qq, kk, vv, gg):
+        return (orc.linattn_bidirectional(qq, kk, vv, grid, split, heads, gate=gg)[0] * dy).sum()
+
+    h = 1e-6
+    names = ["q", "k", "v"] + (["g"] if gated else [])
+    for name, grad in zip(names, grads):
+        u = rand(B, N, C)
+        args = dict(qq=q, kk=k, vv=v, gg=g)
+        key = name * 2
+        x = args[key]
+        args[key] = x + h * u
+        lp = loss(**args)
+        args[key] = x - h * u
+        lm = loss(**args)
+        fd = (lp - lm) / (2 * h)
+        assert abs(fd - (grad * u).sum()) <= 1e-7 * max(1.0, abs(fd)), (name, fd, (grad * u).sum())
+    assert grads[3] is None or gated
+
+
+def test_backward_of_v_is_linear_and_ignores_the_gate_scale_of_q():
+    """dV = K'^T-weighted sum of dnum (the layer is linear in V): scaling dY
+    scales every gradient; dV equals the finite difference exactly for a
+    linear layer even with a large step."""
+    grid, split, heads, D = (2, 2, 3), (1, 1, 2), 1, 8
+    N = 12
+    q, k, v, dy = (rand(1, N, D) for _ in range(4))
+    g1 = orc.linattn_backward(q, k, v, grid, split, heads, dy)
+    g2 = orc.linattn_backward(q, k, v, grid, split, heads, 3.0 * dy)
+    for a, b in zip(g1[:3], g2[:3]):
+        assert rel(3.0 * a, b) < 1e-14
+    u = rand(1, N, D)
+    y0 = orc.linattn_bidirectional(q, k, v, grid, split, heads)[0]
+    y1 = orc.linattn_bidirectional(q, k, v + 10.0 * u, grid, split, heads)[0]
+    assert abs(((y1 - y0) * dy).sum() / 10.0 - (g1[2] * u).sum()) < 1e-10
+
+
 def test_token_recurrence_equals_prefix_recomputation():
     """Chunk size 1 token: the sec. 3.4 recurrence = brute force with j <= i."""
     grid, split, heads = (2, 3, 4), (2, 1, 1), 2
