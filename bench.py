@@ -542,6 +542,24 @@ def run_scan_only(args):
                       "GB_per_s": nb / (ms / 1e3) / 1e9}), flush=True)
 
 
+def run_bwd_only(args):
+    """Backward of the gated linear-attention layer at 720p/5s (dq, dk, dv, dg
+    from dy; S and z recomputed): K steps, ms per call."""
+    import softmax_attention_sana_b200 as sana
+    q, k, v, g = (t.cuda() for t in si.qkvg(WL))
+    dy = si.normal(7000, (1, WL.N, WL.C)).cuda()
+    grid = (WL.T, WL.H, WL.W)
+    rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
+    f = lambda: sana.linattn_bwd(q, k, v, g, rope, grid, WL.heads, dy)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    nb = 9 * TENSOR_BYTES  # q, k, v, g, dy read once; dq, dk, dv, dg written once
+    print(json.dumps({"linattn_bwd_720p_ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
+                      "GB_per_s": nb / (ms / 1e3) / 1e9}), flush=True)
+
+
 def run_sparse_only(args):
     """The block-sparse anchor on the 720p/5s grid, a quarter of the key tiles
     per 256-query block (selection included): K steps, ms per call."""
@@ -586,6 +604,8 @@ def main():
                     help="run only the 480p-shaped softmax anchor (a small case for profiling)")
     ap.add_argument("--scan-only", action="store_true",
                     help="run only the whole-sequence block-causal scan at 720p/60s")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="run only the linear-attention backward at 720p/5s")
     ap.add_argument("--sparse-only", action="store_true",
                     help="run only the block-sparse anchor at 720p/5s (25%% of the key tiles)")
     args = ap.parse_args()
@@ -602,6 +622,9 @@ def main():
             return
         if args.sparse_only:
             run_sparse_only(args)
+            return
+        if args.bwd_only:
+            run_bwd_only(args)
             return
         if args.impl == "reference":
             run_reference(args, world, rank)

@@ -136,6 +136,24 @@ SANA_API sana_status sana_linattn_apply(const sana_shape* shape, sana_dtype dtyp
                                         sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward of sana_linattn_fwd ([SV1] sec. 3.2 forward; the pages train the
+ * model from scratch but print no backward: this is the chain rule through the
+ * forward as written, with ReLU'(x) = 1 for x > 0 and 0 otherwise).
+ * Given dy = dL/dY, writes dq, dk, dv (and d_gate when gate_logits is given;
+ * both NULL for the ungated layer), all device (B, N, C) bf16, overwritten.
+ * (S, z) are recomputed from k, v.  bf16 only (head_dim 128).  Workspace:
+ * sana_linattn_bwd_workspace_size() bytes (split partials and combined S, z,
+ * dS, dz; 256-byte aligned).  Gradients must not alias inputs or each other.
+ * Deterministic: every reduction runs in a fixed order.
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_linattn_bwd_workspace_size(const sana_shape* shape, sana_dtype dtype);
+SANA_API sana_status sana_linattn_bwd(const sana_shape* shape, sana_dtype dtype, const void* q,
+                                      const void* k, const void* v, const void* gate_logits,
+                                      const sana_rope* rope, float eps, const void* dy, void* dq,
+                                      void* dk, void* dv, void* d_gate, void* ws, size_t ws_bytes,
+                                      sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * One block of block-causal linear attention with the constant-memory state
  * ([SV1] sec. 3.4 causal O_i and Algorithm 1).  shape describes the chunk
  * (its T frames starting at absolute frame shape->t_offset).  The chunk's own

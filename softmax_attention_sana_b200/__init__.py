@@ -6,7 +6,7 @@ csrc/); this package is a thin ctypes binding over it.
 
 from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_route, check,
                    gemm_bf16, host_rope_tables, hybrid_stack_fwd, last_error, lib,
-                   linattn_apply, linattn_block_causal_scan, linattn_block_causal_scan_workspace_size,
+                   linattn_apply, linattn_bwd, linattn_block_causal_scan, linattn_block_causal_scan_workspace_size,
                    linattn_block_causal_step, linattn_fwd, linattn_state,
                    linattn_workspace_size, rmsnorm,
                    anchor_tile_count, softmax_anchor_fwd, softmax_anchor_sparse_fwd,
@@ -16,7 +16,7 @@ from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_ro
 __all__ = [
     "EPI_NONE", "EPI_RESIDUAL", "EPI_SILU", "Rope", "SanaError", "attnres_route", "check",
     "gemm_bf16", "host_rope_tables", "hybrid_stack_fwd", "last_error", "lib",
-    "linattn_apply", "linattn_block_causal_scan", "linattn_block_causal_scan_workspace_size",
+    "linattn_apply", "linattn_bwd", "linattn_block_causal_scan", "linattn_block_causal_scan_workspace_size",
     "linattn_block_causal_step", "linattn_fwd", "linattn_state", "linattn_workspace_size", "rmsnorm",
     "anchor_tile_count", "softmax_anchor_fwd", "softmax_anchor_sparse_fwd",
     "softmax_anchor_sparse_workspace_size", "stack_config",

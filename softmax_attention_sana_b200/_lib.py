@@ -85,6 +85,10 @@ def _load():
                                                    c_void_p, c_void_p, POINTER(RopeStruct),
                                                    c_float, c_void_p, c_void_p, c_int, c_void_p,
                                                    c_void_p, c_size_t, c_void_p]),
+        "sana_linattn_bwd_workspace_size": (c_size_t, [POINTER(Shape), c_int]),
+        "sana_linattn_bwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     POINTER(RopeStruct), c_float, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
         "sana_softmax_anchor_workspace_size": (c_size_t, [POINTER(Shape), c_int]),
         "sana_softmax_anchor_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, POINTER(RopeStruct), c_float, c_void_p,
@@ -264,6 +268,25 @@ def linattn_block_causal_step(q, k, v, gate, rope: Rope, grid, t_offset, heads, 
         ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(rope.struct), eps,
         _ptr(state_S), _ptr(state_z), int(bool(commit)), _ptr(out), _ptr(ws), ws.numel(), _stream()))
     return out
+
+
+def linattn_bwd(q, k, v, gate, rope: Rope, grid, heads, dy, eps=1e-6, ws=None):
+    """Gradients (dq, dk, dv, dgate) of the gated linear-attention layer for dY
+    (dgate is None for the ungated layer).  bf16."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dy, "dy")):
+        _need(t, n)
+    B, N, C = q.shape
+    D = C // heads
+    dt = _dtype_code(q)
+    s = make_shape(B, grid, heads, D)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = None if gate is None else torch.empty_like(gate)
+    if ws is None:
+        ws = _ws(lib.sana_linattn_bwd_workspace_size(ctypes.byref(s), dt), q.device)
+    check(lib.sana_linattn_bwd(
+        ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(rope.struct), eps,
+        _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(), _stream()))
+    return dq, dk, dv, dg
 
 
 def linattn_block_causal_scan_workspace_size(B, grid, heads, D, chunk_frames, dtype_code,

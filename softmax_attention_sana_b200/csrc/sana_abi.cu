@@ -292,6 +292,36 @@ sana_status linattn_apply_run(const sana_shape& s, sana_dtype dt, const void* q,
   return apply_phase(s, dt, q, gt, rope, g, S, z, eps, out, st);
 }
 
+// ---------------------------------------------------------------- backward (bf16)
+// Workspace: the forward state phase's partials and combined (S, z), then the
+// same again for (dS, dz).
+size_t linattn_bwd_ws_bytes(const sana_shape& s) {
+  const size_t one = carve_linattn(s, SANA_BF16, nullptr).bytes;
+  return 2 * one;
+}
+
+sana_status linattn_bwd_run(const sana_shape& s, const void* q, const void* k, const void* v,
+                            const void* gt, const void* dy, const RopeDev& rope, float eps,
+                            void* dq, void* dk, void* dv, void* dg, void* ws, size_t ws_bytes,
+                            cudaStream_t st) {
+  const GridDev g = to_grid(s);
+  if (g.N == 0) return SANA_OK;
+  const size_t one = carve_linattn(s, SANA_BF16, nullptr).bytes;
+  if (ws_bytes < 2 * one)
+    return fail(SANA_ERR_WORKSPACE, "linear attention backward: workspace %zu < %zu bytes",
+                ws_bytes, 2 * one);
+  if (rope_smem_bytes(g, rope) > kRopeSmemMax)
+    return fail(SANA_ERR_UNSUPPORTED, "linear attention backward: grid needs too many RoPE table bytes");
+  const LinWs fw = carve_linattn(s, SANA_BF16, ws);
+  const LinWs bw = carve_linattn(s, SANA_BF16, static_cast<char*>(ws) + one);
+  const LinAttnPlan plan = linattn_plan(s, SANA_BF16);
+  if (sana_status e = linattn_bf16_state(s, plan, k, v, rope, g, nullptr, nullptr, nullptr, nullptr,
+                                         fw.ws_S, fw.ws_z, fw.S_f32, fw.z_comb, st))
+    return e;
+  return linattn_bf16_backward(s, plan, q, k, v, gt, dy, rope, g, eps, fw.S_f32, fw.z_comb,
+                               bw.ws_S, bw.ws_z, bw.S_f32, bw.z_comb, dq, dk, dv, dg, st);
+}
+
 // ---------------------------------------------------------------- anchor
 sana_status rope_rotate_run(const void* x, bool bf16, const RopeDev* rope, const GridDev& g, int B,
                             int D, float mul, void* out, cudaStream_t st);
@@ -487,6 +517,47 @@ sana_status sana_linattn_block_causal_step(const sana_shape* s, sana_dtype dt, c
                                            sana_stream_t stream) {
   return linattn_common("sana_linattn_block_causal_step", s, dt, q, k, v, g, rope, eps, S, z, true,
                         commit, out, ws, ws_bytes, stream);
+}
+
+size_t sana_linattn_bwd_workspace_size(const sana_shape* s, sana_dtype dt) {
+  if (check_shape(s, dt, "sana_linattn_bwd_workspace_size") != SANA_OK || dt != SANA_BF16) return 0;
+  return linattn_bwd_ws_bytes(*s);
+}
+
+sana_status sana_linattn_bwd(const sana_shape* s, sana_dtype dt, const void* q, const void* k,
+                             const void* v, const void* g, const sana_rope* rope, float eps,
+                             const void* dy, void* dq, void* dk, void* dv, void* dg, void* ws,
+                             size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_linattn_bwd";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (dt != SANA_BF16) return fail(SANA_ERR_UNSUPPORTED, "%s: bf16 only", who);
+  if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!std::isfinite(eps) || eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", who);
+  if (s->T == 0) return SANA_OK;
+  if (!q || !k || !v || !dy || !dq || !dk || !dv)
+    return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  if ((g == nullptr) != (dg == nullptr))
+    return fail(SANA_ERR_INVALID_ARG, "%s: gate_logits and d_gate must both be given or both be NULL", who);
+  const void* ins[5] = {q, k, v, g, dy};
+  const void* outs[4] = {dq, dk, dv, dg};
+  for (const void* p : ins)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  for (const void* p : outs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * 2;
+  for (const void* o : outs) {
+    for (const void* i : ins)
+      if (overlap(o, n, i, n)) return fail(SANA_ERR_INVALID_ARG, "%s: a gradient aliases an input", who);
+    for (const void* o2 : outs)
+      if (o2 != o && overlap(o, n, o2, n)) return fail(SANA_ERR_INVALID_ARG, "%s: gradients alias each other", who);
+  }
+  const size_t need = linattn_bwd_ws_bytes(*s);
+  if (!ws || ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  return linattn_bwd_run(*s, q, k, v, g, dy, to_dev(*rope), eps, dq, dk, dv, dg, ws, ws_bytes,
+                         stream);
 }
 
 size_t sana_linattn_block_causal_scan_workspace_size(const sana_shape* s, int chunk_frames,

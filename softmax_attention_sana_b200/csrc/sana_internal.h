@@ -119,6 +119,23 @@ sana_status linattn_f32_apply(const sana_shape& s, const float* q, const float* 
                               const float* z, float eps, float* out, cudaStream_t st);
 
 
+// Fixed-order sum of split partials (+ an optional carried state), any D.
+void launch_linattn_combine(int BH, const float* ws_S, const float* ws_z, int splits, int D,
+                            const float* S_prev, const float* z_prev, float* S_state,
+                            float* z_state, float* S_f32, float* z_out, cudaStream_t st);
+// Backward of the bf16 layer given S, z (linattn_bwd_tc.cu).
+sana_status linattn_bf16_backward(const sana_shape& s, const LinAttnPlan& plan, const void* q,
+                                  const void* k, const void* v, const void* gt, const void* dy,
+                                  const RopeDev& rope, const GridDev& g, float eps,
+                                  const float* S, const float* z, float* ws_dS, float* ws_dz,
+                                  float* dS, float* dz, void* dq, void* dk, void* dv, void* dg,
+                                  cudaStream_t st);
+size_t linattn_bwd_ws_bytes(const sana_shape& s);
+sana_status linattn_bwd_run(const sana_shape& s, const void* q, const void* k, const void* v,
+                            const void* gt, const void* dy, const RopeDev& rope, float eps,
+                            void* dq, void* dk, void* dv, void* dg, void* ws, size_t ws_bytes,
+                            cudaStream_t st);
+
 // Bidirectional (S_prev == nullptr) or block-causal step.
 sana_status linattn_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,
                         const void* v, const void* g, const RopeDev& rope, float eps,

@@ -160,6 +160,23 @@ def test_sparse_anchor_sizes_and_validation():
     assert call(ws_bytes=64) == L.SANA_ERR_WORKSPACE
 
 
+def test_backward_validation():
+    L = _lib
+    s = _shape(head_dim=128)
+    assert L.lib.sana_linattn_bwd_workspace_size(ctypes.byref(s), L.SANA_BF16) > 0
+    assert L.lib.sana_linattn_bwd_workspace_size(ctypes.byref(_shape()), L.SANA_F32) == 0
+    r = _lib.RopeStruct(16, 16, 16, 16, 16, 16, 22, 21, 21, 2, 4, 4)
+    M = 1 << 20
+
+    def call(dtype=L.SANA_BF16, g=None, dg=None, dq=5 * M, ws_bytes=1 << 26):
+        return L.lib.sana_linattn_bwd(ctypes.byref(s), dtype, M, 2 * M, 3 * M, g, ctypes.byref(r),
+                                      1e-6, 4 * M, dq, 6 * M, 7 * M, dg, 1 << 28, ws_bytes, None)
+    assert call(dtype=L.SANA_F32) == L.SANA_ERR_UNSUPPORTED
+    assert call(g=8 * M) == L.SANA_ERR_INVALID_ARG and "d_gate" in L.last_error()
+    assert call(dq=2 * M) == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
+    assert call(ws_bytes=64) == L.SANA_ERR_WORKSPACE
+
+
 def test_attnres_and_gemm_validation():
     L = _lib
     arr = (ctypes.c_void_p * 1)(4096)
