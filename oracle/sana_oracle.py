@@ -480,6 +480,31 @@ def attnres_route(sources, w, eps=RMS_EPS):
     return h, alpha
 
 
+def attnres_route_backward(sources, w, dh, eps=RMS_EPS):
+    """Gradients of attnres_route's h with respect to the sources and w, given
+    dh: the chain rule through the forward as written (the pages print no
+    backward).  With r_i = sqrt(mean_c v_i^2 + eps) and l_i = w . v_i / r_i:
+      d alpha_i = dh . v_i,  d l_i = alpha_i (d alpha_i - sum_j alpha_j d alpha_j),
+      d v_i = alpha_i dh + d l_i (w / r_i - l_i v_i / (C r_i^2)),
+      d w = sum over tokens of sum_i d l_i v_i / r_i.
+    Returns (list of d v_i, d w)."""
+    V = np.stack([np.asarray(s, np.float64) for s in sources], axis=-2)  # B,N,S,C
+    w = np.asarray(w, np.float64)
+    dh = np.asarray(dh, np.float64)
+    C = V.shape[-1]
+    r = np.sqrt(np.mean(V * V, axis=-1) + eps)                          # B,N,S
+    logits = (V @ w) / r
+    m = logits.max(axis=-1, keepdims=True)
+    e = np.exp(logits - m)
+    alpha = e / e.sum(axis=-1, keepdims=True)
+    dalpha = np.einsum('bnc,bnsc->bns', dh, V)
+    dl = alpha * (dalpha - (alpha * dalpha).sum(axis=-1, keepdims=True))
+    dV = (alpha[..., None] * dh[..., None, :]
+          + dl[..., None] * (w / r[..., None] - (logits / (C * r * r))[..., None] * V))
+    dw = np.einsum('bns,bnsc->c', dl / r, V)
+    return [dV[..., i, :] for i in range(V.shape[-2])], dw
+
+
 # --------------------------------------------------------------------------
 # hybrid stack ([SV2] method paragraph; [SV2-abs] 3:1 interleave)
 # --------------------------------------------------------------------------

@@ -467,6 +467,30 @@ def test_tile_restricted_anchor_equals_dense_when_all_kept_and_gathered_softmax(
 
 # ------------------------------------------------------------------ AttnRes (P6)
 
+@pytest.mark.parametrize("S,C", [(1, 8), (2, 16), (3, 24), (4, 8)])
+def test_attnres_backward_matches_central_finite_differences(S, C):
+    B, N = 2, 5
+    srcs = [rand(B, N, C) * (1 + i) for i in range(S)]
+    w = rand(C)
+    dh = rand(B, N, C)
+    d_srcs, dw = orc.attnres_route_backward(srcs, w, dh)
+
+    def loss(ss, ww):
+        return (orc.attnres_route(ss, ww)[0] * dh).sum()
+
+    h = 1e-6
+    for i in range(S):
+        u = rand(B, N, C)
+        plus = [x + h * u if j == i else x for j, x in enumerate(srcs)]
+        minus = [x - h * u if j == i else x for j, x in enumerate(srcs)]
+        fd = (loss(plus, w) - loss(minus, w)) / (2 * h)
+        assert abs(fd - (d_srcs[i] * u).sum()) <= 1e-7 * max(1.0, abs(fd)), (i, fd)
+    u = rand(C)
+    fd = (loss(srcs, w + h * u) - loss(srcs, w - h * u)) / (2 * h)
+    assert abs(fd - (dw * u).sum()) <= 1e-7 * max(1.0, abs(fd))
+    if S == 1:  # one source: h = v, so dv = dh and dw = 0
+        assert rel(d_srcs[0], dh) < 1e-14 and np.abs(dw).max() < 1e-12
+
 def test_attnres_two_source_closed_form():
     """C = 4, v1 = a e1 (a > 0), v2 = 0.  RMSNorm(v1) = a e1 / sqrt(a^2/4 + eps),
     RMSNorm(0) = 0.  With w = (L, 0, 0, 0) the logits are
