@@ -330,7 +330,27 @@ def components(sana, args):
         f()
     ms = time_loop(f, 20)
     out["attnres_route_720p_3src"] = {"ms": ms, "GB_per_s": 4 * TENSOR_BYTES / (ms / 1e3) / 1e9}
-    del srcs, h
+    # its backward: 3 sources and dh read, 3 source gradients written, dw summed
+    dh = si.normal(7100, (1, si.P720.N, si.P720.C)).cuda()
+    wsb = torch.empty(sana._lib.lib.sana_attnres_route_bwd_workspace_size(1, si.P720.N, si.P720.C),
+                      dtype=torch.uint8, device="cuda")
+    f = lambda: sana.attnres_route_bwd(srcs, w_attn, dh, ws=wsb)
+    for _ in range(3):
+        f()
+    ms = time_loop(f, 20)
+    out["attnres_route_bwd_720p_3src"] = {"ms": ms, "GB_per_s": 7 * TENSOR_BYTES / (ms / 1e3) / 1e9}
+    del srcs, h, dh, wsb
+    # backward of the gated linear-attention layer (S, z recomputed)
+    q, k, v, g = (t.cuda() for t in si.qkvg(WL))
+    dy = si.normal(7000, (1, WL.N, WL.C)).cuda()
+    rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
+    f = lambda: sana.linattn_bwd(q, k, v, g, rope, (WL.T, WL.H, WL.W), WL.heads, dy)
+    for _ in range(3):
+        f()
+    ms = time_loop(f, 20)
+    out["linattn_bwd_720p"] = {"ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
+                               "GB_per_s": 9 * TENSOR_BYTES / (ms / 1e3) / 1e9}
+    del q, k, v, g, dy
     # projection GEMM of the stack: QKVG at 720p, (75,600 x 3072) . (12,288 x 3072)^T
     A = torch.randn(WL.N, WL.C, device="cuda", dtype=torch.bfloat16)
     Wq = torch.randn(4 * WL.C, WL.C, device="cuda", dtype=torch.bfloat16) * WL.C ** -0.5

@@ -259,6 +259,23 @@ SANA_API sana_status sana_attnres_route(int B, long long N, int C, sana_dtype dt
                                sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward of sana_attnres_route ([SV2] AttnRes equation; the pages print no
+ * backward: the chain rule through the route as written).  Given dh = dL/dh
+ * (device (B, N, C) bf16) writes d_sources[i] = dL/dv_i (HOST array of
+ * num_sources device pointers, each (B, N, C) bf16, overwritten) and
+ * dw = dL/dw (device fp32 (C), overwritten; summed over all tokens in a fixed
+ * order, bit-reproducible).  bf16 only; 1 <= num_sources <= 4; C a multiple of
+ * 256 up to 4096.  Workspace: sana_attnres_route_bwd_workspace_size() bytes
+ * (per-CTA partial sums of dw).
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_attnres_route_bwd_workspace_size(int B, long long N, int C);
+SANA_API sana_status sana_attnres_route_bwd(int B, long long N, int C, sana_dtype dtype,
+                                            const void* const* sources, int num_sources,
+                                            const float* w, float rms_eps, const void* dh,
+                                            void* const* d_sources, float* dw, void* ws,
+                                            size_t ws_bytes, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Building blocks of the stack, exported for stage-wise checking.
  * sana_gemm_bf16: out[M][N] = epilogue(A[M][K] . W[N][K]^T) with bf16 A, W, out
  * and fp32 accumulation on tcgen05; epilogue 0 = identity, 1 = SiLU,

@@ -4,7 +4,8 @@ The compute lives in libsana.so (C ABI declared in include/sana.h, kernels in
 csrc/); this package is a thin ctypes binding over it.
 """
 
-from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_route, check,
+from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_route,
+                   attnres_route_bwd, check,
                    gemm_bf16, host_rope_tables, hybrid_stack_fwd, last_error, lib,
                    linattn_apply, linattn_bwd, linattn_block_causal_scan, linattn_block_causal_scan_workspace_size,
                    linattn_block_causal_step, linattn_fwd, linattn_state,
@@ -14,7 +15,8 @@ from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_ro
                    sync_status)
 
 __all__ = [
-    "EPI_NONE", "EPI_RESIDUAL", "EPI_SILU", "Rope", "SanaError", "attnres_route", "check",
+    "EPI_NONE", "EPI_RESIDUAL", "EPI_SILU", "Rope", "SanaError", "attnres_route",
+    "attnres_route_bwd", "check",
     "gemm_bf16", "host_rope_tables", "hybrid_stack_fwd", "last_error", "lib",
     "linattn_apply", "linattn_bwd", "linattn_block_causal_scan", "linattn_block_causal_scan_workspace_size",
     "linattn_block_causal_step", "linattn_fwd", "linattn_state", "linattn_workspace_size", "rmsnorm",

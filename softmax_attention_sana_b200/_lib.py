@@ -100,6 +100,10 @@ def _load():
                                                    c_void_p, c_size_t, c_void_p]),
         "sana_attnres_route": (c_int, [c_int, c_longlong, c_int, c_int, POINTER(c_void_p), c_int,
                                        c_void_p, c_float, c_void_p, c_void_p, c_void_p]),
+        "sana_attnres_route_bwd_workspace_size": (c_size_t, [c_int, c_longlong, c_int]),
+        "sana_attnres_route_bwd": (c_int, [c_int, c_longlong, c_int, c_int, POINTER(c_void_p),
+                                           c_int, c_void_p, c_float, c_void_p, POINTER(c_void_p),
+                                           c_void_p, c_void_p, c_size_t, c_void_p]),
         "sana_gemm_bf16": (c_int, [c_longlong, c_int, c_int, c_void_p, c_longlong, c_void_p,
                                    c_void_p, c_longlong, c_int, c_void_p]),
         "sana_rmsnorm": (c_int, [c_longlong, c_int, c_int, c_void_p, c_float, c_void_p, c_void_p]),
@@ -393,6 +397,25 @@ def attnres_route(sources, w, rms_eps=1e-6, out=None, alpha=None, want_alpha=Fal
     check(lib.sana_attnres_route(B, N, C, dt, arr, len(sources), _ptr(w), rms_eps, _ptr(out),
                                  _ptr(alpha), _stream()))
     return (out, alpha) if want_alpha else out
+
+
+def attnres_route_bwd(sources, w, dh, rms_eps=1e-6, ws=None):
+    """Gradients (list of d sources, d w) of attnres_route for dh.  bf16 sources."""
+    for i, t in enumerate(sources):
+        _need(t, f"sources[{i}]")
+    _need(w, "w")
+    _need(dh, "dh")
+    B, N, C = sources[0].shape
+    dt = _dtype_code(sources[0])
+    grads = [torch.empty_like(t) for t in sources]
+    dw = torch.empty(C, dtype=torch.float32, device=w.device)
+    if ws is None:
+        ws = _ws(lib.sana_attnres_route_bwd_workspace_size(B, N, C), w.device)
+    src = (c_void_p * len(sources))(*[t.data_ptr() for t in sources])
+    dst = (c_void_p * len(grads))(*[t.data_ptr() for t in grads])
+    check(lib.sana_attnres_route_bwd(B, N, C, dt, src, len(sources), _ptr(w), rms_eps, _ptr(dh),
+                                     dst, _ptr(dw), _ptr(ws), ws.numel(), _stream()))
+    return grads, dw
 
 
 def rmsnorm(x, eps=1e-6, out=None):

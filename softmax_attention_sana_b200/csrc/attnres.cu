@@ -300,6 +300,179 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// ---------------------------------------------------------------- backward
+// Chain rule through the route as written (the pages print no backward):
+//   r_s = sqrt(mean v_s^2 + eps),  l_s = w . v_s / r_s,  alpha = softmax(l),
+//   d alpha_s = dh . v_s,  d l_s = alpha_s (d alpha_s - sum_t alpha_t d alpha_t),
+//   d v_s = alpha_s dh + (d l_s / r_s) w - (d l_s l_s / (C r_s^2)) v_s,
+//   d w = sum over tokens of sum_s (d l_s / r_s) v_s.
+// Warp per token with a fixed token-to-warp assignment; the token's source
+// rows stay in registers between the reductions and the gradient pass.  Each
+// warp adds its share of d w to its own shared-memory row; the CTA writes the
+// fixed-order sum of its rows and attnres_dw_reduce_kernel adds the CTA rows
+// in order, so d w is bit-reproducible.
+constexpr int kBwdWarps = 8;
+
+template <int NS, int CH>
+__global__ void __launch_bounds__(256)
+    attnres_bwd_kernel(SourcePtrs src, const __nv_bfloat16* __restrict__ dh, long long tokens,
+                       int C, const float* __restrict__ w, float eps, SourcePtrs dsrc,
+                       float* __restrict__ dw_part) {
+  extern __shared__ float dw_rows[];  // [kBwdWarps][C]
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* myrow = dw_rows + (size_t)wib * C;
+  for (int i = lane; i < C; i += 32) myrow[i] = 0.f;
+  __syncwarp();
+  const long long nwarps = (long long)gridDim.x * kBwdWarps;
+  const float invC = 1.f / (float)C;
+  for (long long tok = (long long)blockIdx.x * kBwdWarps + wib; tok < tokens; tok += nwarps) {
+    const size_t row = (size_t)tok * C;
+    uint4 x[NS][CH];
+#pragma unroll
+    for (int s = 0; s < NS; ++s)
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = (c * 32 + lane) * 8;
+        x[s][c] = col < C ? *reinterpret_cast<const uint4*>(
+                                static_cast<const __nv_bfloat16*>(src.p[s]) + row + col)
+                          : make_uint4(0, 0, 0, 0);
+      }
+    float ss[NS], sw[NS], sd[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) ss[s] = sw[s] = sd[s] = 0.f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * 32 + lane) * 8;
+      if (col >= C) continue;
+      const float4 w0 = *reinterpret_cast<const float4*>(w + col);
+      const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
+      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      float dv[8];
+      Vec8<__nv_bfloat16> dhc;
+      dhc.load(dh + row + col);
+      dhc.to_float(dv);
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf2_to_f2(u[i]);
+          ss[s] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss[s]));
+          sw[s] = fmaf(wv[2 * i], f.x, fmaf(wv[2 * i + 1], f.y, sw[s]));
+          sd[s] = fmaf(dv[2 * i], f.x, fmaf(dv[2 * i + 1], f.y, sd[s]));
+        }
+      }
+    }
+    float a[NS], l[NS], r[NS], m = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss[s] += __shfl_xor_sync(0xffffffffu, ss[s], o);
+        sw[s] += __shfl_xor_sync(0xffffffffu, sw[s], o);
+        sd[s] += __shfl_xor_sync(0xffffffffu, sd[s], o);
+      }
+      r[s] = sqrtf(ss[s] * invC + eps);
+      l[s] = sw[s] / r[s];
+      m = fmaxf(m, l[s]);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      a[s] = expf(l[s] - m);
+      den += a[s];
+    }
+    float adot = 0.f;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      a[s] /= den;
+      adot = fmaf(a[s], sd[s], adot);
+    }
+    float cw[NS], cv[NS];  // d v_s = a_s dh + cw_s w + cv_s v_s
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const float dl = a[s] * (sd[s] - adot);
+      cw[s] = dl / r[s];
+      cv[s] = -dl * l[s] * invC / (r[s] * r[s]);
+    }
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * 32 + lane) * 8;
+      if (col >= C) continue;
+      const float4 w0 = *reinterpret_cast<const float4*>(w + col);
+      const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
+      const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      float dv[8];
+      Vec8<__nv_bfloat16> dhc;
+      dhc.load(dh + row + col);
+      dhc.to_float(dv);
+      float dwv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
+        float g[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf2_to_f2(u[i]);
+          g[2 * i] = fmaf(cv[s], f.x, fmaf(cw[s], wv[2 * i], a[s] * dv[2 * i]));
+          g[2 * i + 1] = fmaf(cv[s], f.y, fmaf(cw[s], wv[2 * i + 1], a[s] * dv[2 * i + 1]));
+          dwv[2 * i] = fmaf(cw[s], f.x, dwv[2 * i]);
+          dwv[2 * i + 1] = fmaf(cw[s], f.y, dwv[2 * i + 1]);
+        }
+        Vec8<__nv_bfloat16>::store(static_cast<__nv_bfloat16*>(const_cast<void*>(dsrc.p[s])) + row + col, g);
+      }
+      float4* acc = reinterpret_cast<float4*>(myrow + col);
+      const float4 a0 = acc[0], a1 = acc[1];
+      acc[0] = make_float4(a0.x + dwv[0], a0.y + dwv[1], a0.z + dwv[2], a0.w + dwv[3]);
+      acc[1] = make_float4(a1.x + dwv[4], a1.y + dwv[5], a1.z + dwv[6], a1.w + dwv[7]);
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < kBwdWarps; ++k) acc += dw_rows[k * C + c];
+    dw_part[(size_t)blockIdx.x * C + c] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    attnres_dw_reduce_kernel(const float* __restrict__ dw_part, int nblocks, int C,
+                             float* __restrict__ dw) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= C) return;
+  float acc = 0.f;
+  for (int b = 0; b < nblocks; ++b) acc += dw_part[(size_t)b * C + c];
+  dw[c] = acc;
+}
+
+int attnres_bwd_blocks(long long tokens) {
+  const long long want = (tokens + kBwdWarps - 1) / kBwdWarps;
+  const long long cap = kNumSMs;  // one CTA of 8 warps per SM (registers: ~220 per thread at 3 sources)
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+template <int NS, int CH>
+void bwd_launch(const SourcePtrs& sp, const void* dh, long long tokens, int C, const float* w,
+                float eps, const SourcePtrs& dsp, float* dw_part, cudaStream_t st) {
+  const int blocks = attnres_bwd_blocks(tokens);
+  const int smem = kBwdWarps * C * (int)sizeof(float);
+  cudaFuncSetAttribute(attnres_bwd_kernel<NS, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  attnres_bwd_kernel<NS, CH><<<blocks, 256, smem, st>>>(
+      sp, static_cast<const __nv_bfloat16*>(dh), tokens, C, w, eps, dsp, dw_part);
+}
+
+template <int CH>
+void bwd_launch_s(const SourcePtrs& sp, int S, const void* dh, long long tokens, int C,
+                  const float* w, float eps, const SourcePtrs& dsp, float* dw_part, cudaStream_t st) {
+  switch (S) {
+    case 1: bwd_launch<1, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+    case 2: bwd_launch<2, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+    case 3: bwd_launch<3, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+    default: bwd_launch<4, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+  }
+}
+
 int threads_for(int C) {
   int t = ((C / 8) + 31) / 32 * 32;
   return t < 32 ? 32 : t;
@@ -372,6 +545,38 @@ sana_status attnres_run(int B, long long N, int C, sana_dtype dt, const void* co
   if (dt == SANA_BF16) launch_attnres<__nv_bfloat16>(sp, S, tokens, C, w, eps, h, alpha, hn, st);
   else launch_attnres<float>(sp, S, tokens, C, w, eps, h, alpha, hn, st);
   return check_launch("attnres_kernel");
+}
+
+size_t attnres_bwd_ws_bytes(long long tokens, int C) {
+  return align_up((size_t)attnres_bwd_blocks(tokens) * C * sizeof(float), 256);
+}
+
+sana_status attnres_bwd_run(long long tokens, int C, const void* const* sources, int S,
+                            const float* w, float eps, const void* dh, void* const* d_sources,
+                            float* dw, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (S < 1 || S > 4 || C % 256 != 0 || C > 4096)
+    return fail(SANA_ERR_UNSUPPORTED, "attnres backward: %d sources, C=%d (1..4 sources, C a multiple of 256 up to 4096)", S, C);
+  if (tokens == 0) {
+    cudaMemsetAsync(dw, 0, (size_t)C * sizeof(float), st);
+    return check_launch("attnres backward (no tokens)");
+  }
+  if (ws_bytes < attnres_bwd_ws_bytes(tokens, C))
+    return fail(SANA_ERR_WORKSPACE, "attnres backward: workspace %zu < %zu bytes", ws_bytes,
+                attnres_bwd_ws_bytes(tokens, C));
+  SourcePtrs sp{}, dsp{};
+  for (int i = 0; i < S; ++i) {
+    sp.p[i] = sources[i];
+    dsp.p[i] = d_sources[i];
+  }
+  float* dw_part = static_cast<float*>(ws);
+  const int ch = C / 256;
+  if (ch <= 4) bwd_launch_s<4>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  else if (ch <= 8) bwd_launch_s<8>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  else if (ch <= 12) bwd_launch_s<12>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  else bwd_launch_s<16>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  if (sana_status e = check_launch("attnres_bwd_kernel")) return e;
+  attnres_dw_reduce_kernel<<<(C + 255) / 256, 256, 0, st>>>(dw_part, attnres_bwd_blocks(tokens), C, dw);
+  return check_launch("attnres_dw_reduce_kernel");
 }
 
 sana_status rmsnorm_run(long long rows, int C, sana_dtype dt, const void* x, float eps, void* y,

@@ -758,6 +758,46 @@ sana_status sana_attnres_route(int B, long long N, int C, sana_dtype dt, const v
                      nullptr, stream);
 }
 
+size_t sana_attnres_route_bwd_workspace_size(int B, long long N, int C) {
+  if (B < 1 || N < 0 || C < 1) return 0;
+  return attnres_bwd_ws_bytes((long long)B * N, C);
+}
+
+sana_status sana_attnres_route_bwd(int B, long long N, int C, sana_dtype dt,
+                                   const void* const* sources, int num_sources, const float* w,
+                                   float rms_eps, const void* dh, void* const* d_sources,
+                                   float* dw, void* ws, size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_attnres_route_bwd";
+  if (dt != SANA_BF16) return fail(SANA_ERR_UNSUPPORTED, "%s: bf16 only", who);
+  if (B < 1 || N < 0 || C < 1) return fail(SANA_ERR_INVALID_ARG, "%s: bad sizes", who);
+  if (num_sources < 1 || num_sources > 4)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: num_sources=%d (1..4)", who, num_sources);
+  if (!std::isfinite(rms_eps) || rms_eps < 0.f) return fail(SANA_ERR_INVALID_ARG, "%s: bad rms_eps", who);
+  if (!w || !dw) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (N == 0)  // no tokens: dw = 0, nothing else is read or written
+    return attnres_bwd_run(0, C, nullptr, num_sources, w, rms_eps, nullptr, nullptr, dw, nullptr,
+                           0, stream);
+  if (!sources || !d_sources || !dh) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  const size_t n = (size_t)B * N * C * 2;
+  for (int i = 0; i < num_sources; ++i) {
+    if (!sources[i] || !aligned16(sources[i]) || !d_sources[i] || !aligned16(d_sources[i]))
+      return fail(SANA_ERR_INVALID_ARG, "%s: source or gradient %d is NULL or not 16-byte aligned", who, i);
+    if (overlap(d_sources[i], n, dh, n)) return fail(SANA_ERR_INVALID_ARG, "%s: gradient %d aliases dh", who, i);
+    for (int j = 0; j < num_sources; ++j) {
+      if (overlap(d_sources[i], n, sources[j], n))
+        return fail(SANA_ERR_INVALID_ARG, "%s: gradient %d aliases source %d", who, i, j);
+      if (j != i && overlap(d_sources[i], n, d_sources[j], n))
+        return fail(SANA_ERR_INVALID_ARG, "%s: gradients %d and %d alias", who, i, j);
+    }
+  }
+  if (!aligned16(w) || !aligned16(dh)) return fail(SANA_ERR_INVALID_ARG, "%s: w / dh not 16-byte aligned", who);
+  const size_t need = attnres_bwd_ws_bytes((long long)B * N, C);
+  if (!ws || ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  return attnres_bwd_run((long long)B * N, C, sources, num_sources, w, rms_eps, dh, d_sources, dw,
+                         ws, ws_bytes, stream);
+}
+
 sana_status sana_rmsnorm(long long rows, int C, sana_dtype dt, const void* x, float eps, void* y,
                          sana_stream_t stream) {
   if (dt != SANA_F32 && dt != SANA_BF16) return fail(SANA_ERR_INVALID_ARG, "sana_rmsnorm: bad dtype");

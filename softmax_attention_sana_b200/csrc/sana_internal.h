@@ -175,6 +175,10 @@ sana_status anchor_sparse_run(const sana_shape& s, const void* q, const void* k,
 sana_status attnres_run(int B, long long N, int C, sana_dtype dt, const void* const* sources,
                         int S, const float* w, float eps, void* h, float* alpha, bool normed_out,
                         void* h_norm, cudaStream_t st);
+size_t attnres_bwd_ws_bytes(long long tokens, int C);
+sana_status attnres_bwd_run(long long tokens, int C, const void* const* sources, int S,
+                            const float* w, float eps, const void* dh, void* const* d_sources,
+                            float* dw, void* ws, size_t ws_bytes, cudaStream_t st);
 sana_status rmsnorm_run(long long rows, int C, sana_dtype dt, const void* x, float eps, void* y,
                         cudaStream_t st);
 sana_status gemm_run(long long M, int N, int K, const void* A, long long lda, const void* W,
