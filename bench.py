@@ -402,13 +402,16 @@ def components(sana, args):
     if args.stacks:
         grid = (WL.T, WL.H, WL.W)
         rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
-        for name, layers, attnres, ffn in (("stack_720p_group4", 4, False, 0),
-                                            ("stack_720p_attnres16", 16, True, 3)):
+        keep = (sana.anchor_tile_count(WL.N) + 3) // 4
+        for name, layers, attnres, ffn, kt in (("stack_720p_group4", 4, False, 0, 0),
+                                                ("stack_720p_group4_sparse25", 4, False, 0, keep),
+                                                ("stack_720p_attnres16", 16, True, 3, 0)):
             x = si.normal(5000 + layers, (1, WL.N, WL.C)).cuda()
             ws_l = [{k2: t.cuda() for k2, t in d.items()}
                     for d in si.projection_weights(5, layers, WL.C, ffn)]
             w_attn, w_ffn = (t.cuda() for t in si.router_queries(5, WL.C))
-            cfg = sana.stack_config(layers, block_span=8, use_attnres=attnres, ffn_mult=ffn)
+            cfg = sana.stack_config(layers, block_span=8, use_attnres=attnres, ffn_mult=ffn,
+                                    anchor_keep_tiles=kt)
             y = torch.empty_like(x)
             f = lambda: sana.hybrid_stack_fwd(x, ws_l, w_attn, w_ffn, rope, grid, WL.heads, cfg, out=y)
             f()
@@ -417,9 +420,13 @@ def components(sana, args):
             lin = 4 * WL.N * WL.heads * WL.D ** 2
             proj = 2 * WL.N * WL.C * WL.C * (4 + 1 + 2 * ffn)
             nanc = layers // 4
+            if kt:  # executed anchor work of the kept tiles
+                nan = 4 * WL.N * min(WL.N, kt * 128) * WL.heads * WL.D
             flops = nanc * nan + (layers - nanc) * lin + layers * proj
             out[name] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12, "layers": layers,
                          "attnres": attnres, "ffn_mult": ffn}
+            if kt:
+                out[name]["anchor_keep_tiles"] = kt
             del x, ws_l, y
     return out
 

@@ -312,6 +312,9 @@ typedef struct {
   float eps;          /* linear-attention denominator eps */
   float rms_eps;      /* RMSNorm eps (routing and pre-norm) */
   float anchor_scale; /* <= 0: 1/sqrt(D) */
+  int anchor_keep_tiles; /* 0: dense anchors; k > 0: block-sparse anchors keeping
+                            the k highest-scoring 128-key tiles per 256-query
+                            block (sana_softmax_anchor_sparse_fwd's selection) */
 } sana_stack_config;
 
 typedef struct {

@@ -518,11 +518,14 @@ def is_anchor_layer(l, ratio=4):
     return l % ratio == ratio - 1
 
 
-def _attention_sublayer(xh, Wl, grid, rope_split, heads, eps, anchor):
+def _attention_sublayer(xh, Wl, grid, rope_split, heads, eps, anchor, anchor_keep=0):
     C = xh.shape[-1]
     qkvg = xh @ np.asarray(Wl['qkvg'], np.float64).T
     q, k, v, g = (qkvg[..., i * C:(i + 1) * C] for i in range(4))
-    if anchor:
+    if anchor and anchor_keep > 0:
+        tiles = anchor_block_select(anchor_block_scores(q, k, grid, rope_split, heads), anchor_keep)
+        a = softmax_anchor_tiles(q, k, v, grid, rope_split, heads, tiles, gate=g)
+    elif anchor:
         a = softmax_anchor(q, k, v, grid, rope_split, heads, gate=g)
     else:
         a, _, _ = linattn_bidirectional(q, k, v, grid, rope_split, heads, gate=g, eps=eps)
@@ -536,7 +539,7 @@ def _ffn_sublayer(xh, Wl):
 
 def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
                  block_span=8, ratio=4, use_attnres=True, ffn=True, eps=EPS,
-                 rms_eps=RMS_EPS):
+                 rms_eps=RMS_EPS, anchor_keep=0):
     """Forward of the hybrid stack.
 
     With AttnRes: every sublayer reads h = route(V_l) over [embedding,
@@ -544,13 +547,14 @@ def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
     the partial sum, and after every block_span layers the partial sum is
     frozen as a block summary.  The result is the representation a next layer
     would read: route(V, w_attn) over the final source set.
-    Without AttnRes: plain pre-norm residual x += sublayer(RMSNorm(x))."""
+    Without AttnRes: plain pre-norm residual x += sublayer(RMSNorm(x)).
+    anchor_keep > 0: the anchors are block-sparse (anchor_block_select's tiles)."""
     x = np.asarray(x, np.float64)
     if not use_attnres:
         for l in range(layers):
             Wl = weights[l]
             x = x + _attention_sublayer(rmsnorm(x, rms_eps), Wl, grid, rope_split,
-                                        heads, eps, is_anchor_layer(l, ratio))
+                                        heads, eps, is_anchor_layer(l, ratio), anchor_keep)
             if ffn:
                 x = x + _ffn_sublayer(rmsnorm(x, rms_eps), Wl)
         return x
@@ -564,7 +568,7 @@ def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
         Wl = weights[l]
         h, _ = attnres_route(sources(), w_attn, rms_eps)
         out = _attention_sublayer(rmsnorm(h, rms_eps), Wl, grid, rope_split, heads,
-                                  eps, is_anchor_layer(l, ratio))
+                                  eps, is_anchor_layer(l, ratio), anchor_keep)
         partial = out if partial is None else partial + out
         if ffn:
             h, _ = attnres_route(sources(), w_ffn, rms_eps)

@@ -46,7 +46,7 @@ class RopeStruct(Structure):
 class StackConfig(Structure):
     _fields_ = [("layers", c_int), ("block_span", c_int), ("ratio", c_int), ("use_attnres", c_int),
                 ("ffn_mult", c_int), ("eps", c_float), ("rms_eps", c_float),
-                ("anchor_scale", c_float)]
+                ("anchor_scale", c_float), ("anchor_keep_tiles", c_int)]
 
 
 class StackWeights(Structure):
@@ -442,9 +442,9 @@ def gemm_bf16(A, W, out=None, epilogue=EPI_NONE):
 # ---------------------------------------------------------------- stack
 
 def stack_config(layers, block_span=8, ratio=4, use_attnres=True, ffn_mult=3, eps=1e-6,
-                 rms_eps=1e-6, anchor_scale=0.0) -> StackConfig:
+                 rms_eps=1e-6, anchor_scale=0.0, anchor_keep_tiles=0) -> StackConfig:
     return StackConfig(layers, block_span, ratio, int(bool(use_attnres)), ffn_mult, eps, rms_eps,
-                       anchor_scale)
+                       anchor_scale, anchor_keep_tiles)
 
 
 def hybrid_stack_fwd(x, weights, w_attn, w_ffn, rope: Rope, grid, heads, cfg: StackConfig,

@@ -37,6 +37,7 @@ struct StackWs {
   std::vector<__nv_bfloat16*> blocks;  // summaries + the running partial sum
   void* attn_ws;
   size_t attn_ws_bytes;
+  int* tiles;  // kept key tiles of the sparse anchors
   size_t bytes;
 };
 
@@ -56,9 +57,14 @@ StackWs carve_stack(const sana_shape& s, const sana_stack_config& c, void* ws) {
     const int nblocks = (c.layers + c.block_span - 1) / c.block_span;
     for (int i = 0; i < nblocks; ++i) w.blocks.push_back(cv.take<__nv_bfloat16>(tok * C));
   }
-  const size_t lin = linattn_ws_bytes(s, SANA_BF16), anc = anchor_ws_bytes(s, SANA_BF16);
+  const size_t lin = linattn_ws_bytes(s, SANA_BF16);
+  const size_t anc = c.anchor_keep_tiles > 0 ? anchor_sparse_ws_bytes(s) : anchor_ws_bytes(s, SANA_BF16);
   w.attn_ws_bytes = lin > anc ? lin : anc;
   w.attn_ws = cv.take<char>(w.attn_ws_bytes);
+  if (c.anchor_keep_tiles > 0) {
+    const size_t ntiles = (tok / s.B + 127) / 128;
+    w.tiles = cv.take<int>((size_t)s.B * s.heads * ((ntiles + 1) / 2) * c.anchor_keep_tiles);
+  }
   w.bytes = align_up(cv.used, 256);
   return w;
 }
@@ -76,6 +82,11 @@ sana_status check_cfg(const sana_shape* s, const sana_stack_config* c) {
   if (c->use_attnres && 1 + (c->layers + c->block_span - 1) / c->block_span > 16)
     return fail(SANA_ERR_UNSUPPORTED, "stack: more than 16 AttnRes sources");
   if (!(c->eps >= 0.f) || !(c->rms_eps >= 0.f)) return fail(SANA_ERR_INVALID_ARG, "stack: bad eps");
+  const long long ntiles = ((long long)s->T * s->H * s->W + 127) / 128;
+  if (c->anchor_keep_tiles < 0 || c->anchor_keep_tiles > ntiles ||
+      (c->anchor_keep_tiles > 0 && ntiles > kAnchorMaxTiles))
+    return fail(SANA_ERR_INVALID_ARG, "stack: anchor_keep_tiles=%d outside [0, %lld]",
+                c->anchor_keep_tiles, ntiles);
   return SANA_OK;
 }
 
@@ -117,9 +128,13 @@ extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_sta
     void* parts[4] = {P.q, P.k, P.v, P.g};
     if (sana_status e = gemm_run_parts(M, 4 * C, C, P.xhat, C, w->w_qkvg[l], parts, 4, C, 0, st))
       return e;
-    if (l % c->ratio == c->ratio - 1)
+    if (l % c->ratio == c->ratio - 1) {
+      if (c->anchor_keep_tiles > 0)
+        return anchor_sparse_run(*s, P.q, P.k, P.v, P.g, &rd, scale, c->anchor_keep_tiles, P.tiles,
+                                 true, P.attn, P.attn_ws, P.attn_ws_bytes, st);
       return anchor_run(*s, SANA_BF16, P.q, P.k, P.v, P.g, &rd, scale, P.attn, P.attn_ws,
                         P.attn_ws_bytes, st);
+    }
     return linattn_run(*s, SANA_BF16, P.q, P.k, P.v, P.g, rd, c->eps, nullptr, nullptr, false,
                        false, P.attn, P.attn_ws, P.attn_ws_bytes, st);
   };

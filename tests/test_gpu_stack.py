@@ -118,10 +118,11 @@ def _run_stack(x, ws, w_attn, w_ffn, grid, heads, cfg):
     return y
 
 
-def _oracle_stack(x, ws, w_attn, w_ffn, grid, heads, layers, span, attnres, ffn):
+def _oracle_stack(x, ws, w_attn, w_ffn, grid, heads, layers, span, attnres, ffn, keep=0):
     wo = [{k: f64(v) for k, v in d.items()} for d in ws]
     return orc.hybrid_stack(f64(x), wo, f64(w_attn), f64(w_ffn), grid, (22, 21, 21), heads,
-                            layers, block_span=span, use_attnres=attnres, ffn=ffn)
+                            layers, block_span=span, use_attnres=attnres, ffn=ffn,
+                            anchor_keep=keep)
 
 
 @pytest.mark.parametrize("layers,span,attnres,ffn", [(4, 8, False, 0), (4, 8, False, 3),
@@ -134,6 +135,22 @@ def test_stack_small_against_oracle(layers, span, attnres, ffn):
     cfg = sana.stack_config(layers, block_span=span, use_attnres=attnres, ffn_mult=ffn)
     y = _run_stack(x, ws, w_attn, w_ffn, grid, heads, cfg)
     yo = _oracle_stack(x, ws, w_attn, w_ffn, grid, heads, layers, span, attnres, ffn > 0)
+    err = orc.max_rel_err(f64(y), yo)
+    assert err <= BF16_TOL, err
+
+
+@pytest.mark.parametrize("keep", [4, 2])
+def test_stack_with_sparse_anchors_against_oracle(keep):
+    """8 layers (2 anchors) on a 4 x 8 x 16 grid (512 tokens: 4 key tiles, 2
+    query blocks): all 4 tiles kept (= dense anchors) and 2 of 4 kept."""
+    grid, heads = (4, 8, 16), 2
+    C, N = 256, 512
+    layers, span = 8, 4
+    x, ws, w_attn, w_ffn = _stack_inputs(C, N, layers, 3, 13100 + keep)
+    cfg = sana.stack_config(layers, block_span=span, use_attnres=True, ffn_mult=3,
+                            anchor_keep_tiles=keep)
+    y = _run_stack(x, ws, w_attn, w_ffn, grid, heads, cfg)
+    yo = _oracle_stack(x, ws, w_attn, w_ffn, grid, heads, layers, span, True, True, keep)
     err = orc.max_rel_err(f64(y), yo)
     assert err <= BF16_TOL, err
 

@@ -465,6 +465,18 @@ def test_tile_restricted_anchor_equals_dense_when_all_kept_and_gathered_softmax(
             assert rel(y[0, ri:ri + 1, sl], yn) < 1e-12
 
 
+def test_stack_with_every_tile_kept_equals_the_dense_stack():
+    grid, split, heads, D = (2, 15, 20), (2, 1, 1), 1, 8
+    N, C, layers = 600, 8, 4
+    x = rand(1, N, C)
+    ws = [{"qkvg": rand(4 * C, C) / np.sqrt(C), "o": rand(C, C) / np.sqrt(C)} for _ in range(layers)]
+    dense = orc.hybrid_stack(x, ws, None, None, grid, split, heads, layers, use_attnres=False,
+                             ffn=False)
+    kept = orc.hybrid_stack(x, ws, None, None, grid, split, heads, layers, use_attnres=False,
+                            ffn=False, anchor_keep=5)
+    assert rel(kept, dense) < 1e-12
+
+
 # ------------------------------------------------------------------ AttnRes (P6)
 
 @pytest.mark.parametrize("S,C", [(1, 8), (2, 16), (3, 24), (4, 8)])
