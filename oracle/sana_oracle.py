@@ -24,7 +24,7 @@ Sources (cited by page title and section / equation):
 * [SV2-abs] "SANA-Video 2.0" abstract (ai-pulse-lab page): gated linear
   attention with gated softmax anchors at a 3:1 ratio.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * 3D RoPE layout: global pair j rotates elements (2j, 2j+1); pairs
   [0, n_t) use the frame index t, the next n_h the row index h, the last n_w
