@@ -48,6 +48,45 @@ __device__ __forceinline__ float2 pair_cs(const RowRope& rr, int j) {
   return rr.cs(j);
 }
 
+// Rotary (cos, sin) of one token read straight from the global tables (the
+// key-side kernel leaves its shared memory to the K/V ring; the tables are
+// small enough to stay in L1).
+struct GlobalRowRope {
+  const float *ct, *st, *ch, *sh, *cw, *sw;
+  int n_t, n_th;
+  __device__ __forceinline__ float2 cs(int j) const {
+    return j < n_t ? make_float2(ct[j], st[j])
+                   : (j < n_th ? make_float2(ch[j - n_t], sh[j - n_t])
+                               : make_float2(cw[j - n_th], sw[j - n_th]));
+  }
+};
+
+__device__ __forceinline__ GlobalRowRope global_row_rope(const RopeDev& r, const GridDev& g,
+                                                         int b, int n) {
+  const int hw = g.H * g.W;
+  const int t = n / hw, rem = n - t * hw, hh = rem / g.W, ww = rem - hh * g.W;
+  const int tt = g.t_offset + b * g.t_stride + t;
+  GlobalRowRope rr;
+  rr.ct = r.cos_t + tt * r.n_t;
+  rr.st = r.sin_t + tt * r.n_t;
+  rr.ch = r.cos_h + hh * r.n_h;
+  rr.sh = r.sin_h + hh * r.n_h;
+  rr.cw = r.cos_w + ww * r.n_w;
+  rr.sw = r.sin_w + ww * r.n_w;
+  rr.n_t = r.n_t;
+  rr.n_th = r.n_t + r.n_h;
+  return rr;
+}
+
+template <int NT, int NH>
+__device__ __forceinline__ float2 pair_cs(const GlobalRowRope& rr, int j) {
+  if (NT >= 0)
+    return j < NT ? make_float2(rr.ct[j], rr.st[j])
+                  : (j < NT + NH ? make_float2(rr.ch[j - NT], rr.sh[j - NT])
+                                 : make_float2(rr.cw[j - NT - NH], rr.sw[j - NT - NH]));
+  return rr.cs(j);
+}
+
 // Rotation by the opposite angle (the transpose of the RoPE rotation).
 __device__ __forceinline__ float2 rotate_t(float x, float y, float2 cs) {
   return make_float2(x * cs.x + y * cs.y, y * cs.x - x * cs.y);
@@ -78,8 +117,8 @@ __device__ void stage_matrix(uint8_t* dst, const float* __restrict__ M, int tid,
 
 // ReLU + RoPE of this thread's 32 columns (quarter C4) of token row r, in
 // place; returns the partial phi(x) . z over those columns and the (x > 0) bits.
-template <int NT, int NH, int C4>
-__device__ __forceinline__ float quarter_forward(uint8_t* tile, int r, const RowRope& rr,
+template <int NT, int NH, int C4, class RR>
+__device__ __forceinline__ float quarter_forward(uint8_t* tile, int r, const RR& rr,
                                                  const float* z, uint32_t& mask) {
   uint8_t* half = tile + (C4 >> 1) * kHalf;
   float den = 0.f;
@@ -109,9 +148,9 @@ __device__ __forceinline__ float quarter_forward(uint8_t* tile, int r, const Row
   return den;
 }
 
-template <int NT, int NH>
+template <int NT, int NH, class RR>
 __device__ __forceinline__ float quarter_forward_any(int c4, uint8_t* tile, int r,
-                                                     const RowRope& rr, const float* z,
+                                                     const RR& rr, const float* z,
                                                      uint32_t& mask) {
   switch (c4) {  // warp-uniform
     case 0: return quarter_forward<NT, NH, 0>(tile, r, rr, z, mask);
@@ -125,8 +164,8 @@ __device__ __forceinline__ float quarter_forward_any(int c4, uint8_t* tile, int 
 // r (quarter C4): grad comes from TMEM in two 16-column parts at tmem_col; the
 // result replaces the tile's row segment.  With zacc, the tile's contents
 // (R phi) are first rotated back and accumulated as add * phi.
-template <int NT, int NH, int C4>
-__device__ __forceinline__ void quarter_backward(uint8_t* tile, int r, const RowRope& rr,
+template <int NT, int NH, int C4, class RR>
+__device__ __forceinline__ void quarter_backward(uint8_t* tile, int r, const RR& rr,
                                                  uint32_t tmem_row, float add, const float* zz,
                                                  uint32_t mask, float* zacc,
                                                  uint64_t* freed) {
@@ -168,9 +207,9 @@ __device__ __forceinline__ void quarter_backward(uint8_t* tile, int r, const Row
   }
 }
 
-template <int NT, int NH>
+template <int NT, int NH, class RR>
 __device__ __forceinline__ void quarter_backward_any(int c4, uint8_t* tile, int r,
-                                                     const RowRope& rr, uint32_t tmem_row,
+                                                     const RR& rr, uint32_t tmem_row,
                                                      float add, const float* zz, uint32_t mask,
                                                      float* zacc, uint64_t* freed) {
   switch (c4) {  // warp-uniform
@@ -537,8 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------
 // key side: dk, dv
 // ------------------------------------------------------------------------
+constexpr int kStagesK = 3;  // k and v rings (they double as dk / dv staging)
+
 struct BwdKCtl {
-  uint64_t fullK[2], fullV[2], kready[2], out_ready[2];
+  uint64_t fullK[kStagesK], fullV[kStagesK], kready[kStagesK], out_ready[kStagesK];
   uint64_t mma_done[2], tmem_free[2];
   uint32_t tmem;
   int abort_flag;
@@ -546,6 +587,8 @@ struct BwdKCtl {
 };
 
 // TMEM columns, per tile parity tb: dk' [256 tb, +128), dv [256 tb + 128, +128).
+// The rotary tables are read from global memory, leaving shared memory to a
+// three-stage K/V ring.
 template <int NT, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
     linattn_bwd_k_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -557,10 +600,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdKCtl ctl;
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* ds_op = smem;               // dS as bf16 [d][e], 32 KB
-  uint8_t* k_st = ds_op + kTileB;      // 2 stages: k -> k' -> dk
-  uint8_t* v_st = k_st + 2 * kTileB;   // 2 stages: v -> dv
-  float2* rope_base = reinterpret_cast<float2*>(v_st + 2 * kTileB);
+  uint8_t* ds_op = smem;                     // dS as bf16 [d][e], 32 KB
+  uint8_t* k_st = ds_op + kTileB;            // k -> k' -> dk
+  uint8_t* v_st = k_st + kStagesK * kTileB;  // v -> dv
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -570,13 +612,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wc{&ctl.abort_flag, status};
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&ctl.fullK[s], 1);
       mbar_init(&ctl.fullV[s], 1);
       mbar_init(&ctl.kready[s], kWorkers);
       mbar_init(&ctl.out_ready[s], kWorkers);
-      mbar_init(&ctl.mma_done[s], 1);
-      mbar_init(&ctl.tmem_free[s], kWorkers);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl.mma_done[t], 1);
+      mbar_init(&ctl.tmem_free[t], kWorkers);
     }
     ctl.abort_flag = 0;
     mbar_fence_init();
@@ -590,7 +634,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     stage_matrix(ds_op, dS_all + (size_t)bh * kD * kD, tid, kWorkers);
     fence_proxy_async_smem();
   }
-  const RopeSmem rs = rope_stage(rope_base, rope, g, b, tid, kThreads);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -603,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_v);
       int issued = 0;
       auto load = [&](int it) {
-        const int s = it & 1, n0 = (tile0 + it) * kRows;
+        const int s = it % kStagesK, n0 = (tile0 + it) * kRows;
         mbar_arrive_expect_tx(&ctl.fullK[s], kTileB);
         tma_load_3d(k_st + s * kTileB, &tm_k, &ctl.fullK[s], h * kD, n0, b);
         tma_load_3d(k_st + s * kTileB + kHalf, &tm_k, &ctl.fullK[s], h * kD + 64, n0, b);
@@ -612,12 +655,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(v_st + s * kTileB + kHalf, &tm_v, &ctl.fullV[s], h * kD + 64, n0, b);
         ++issued;
       };
-      if (ntiles > 0) load(0);
-      if (ntiles > 1) load(1);
+      for (int it = 0; it < kStagesK && it < ntiles; ++it) load(it);
       bool ok = true;
       for (int it = 0; it < ntiles; ++it) {
-        const int s = it & 1, n0 = (tile0 + it) * kRows;
-        if (!mbar_wait(&ctl.out_ready[s], (it >> 1) & 1, wc, 0x61)) {
+        const int s = it % kStagesK, n0 = (tile0 + it) * kRows;
+        if (!mbar_wait(&ctl.out_ready[s], (it / kStagesK) & 1, wc, 0x61)) {
           ok = false;
           break;
         }
@@ -627,13 +669,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_store_3d(&tm_dv, v_st + s * kTileB + kHalf, h * kD + 64, n0, b);
         bulk_commit();
         bulk_wait_read0();
-        if (it + 2 < ntiles) load(it + 2);
+        if (it + kStagesK < ntiles) load(it + kStagesK);
       }
       bulk_wait0();
       if (!ok)
-        for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it) {
-          mbar_drain(&ctl.fullK[it & 1], (it >> 1) & 1);
-          mbar_drain(&ctl.fullV[it & 1], (it >> 1) & 1);
+        for (int it = issued > kStagesK ? issued - kStagesK : 0; it < issued; ++it) {
+          mbar_drain(&ctl.fullK[it % kStagesK], (it / kStagesK) & 1);
+          mbar_drain(&ctl.fullV[it % kStagesK], (it / kStagesK) & 1);
         }
     }
   } else if (warp == kWarpMma) {
@@ -648,8 +690,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t ds_k = smem_desc_sw128(smem_u32(ds_op), 16, 1024);
       const uint64_t ds_m = smem_desc_sw128(smem_u32(ds_op), kHalf, 1024);
       for (int it = 0; it < ntiles; ++it) {
-        const int s = it & 1, tb = it & 1;
-        if (!mbar_wait(&ctl.fullV[s], (it >> 1) & 1, wc, 0x62)) break;
+        const int s = it % kStagesK, tb = it & 1;
+        if (!mbar_wait(&ctl.fullV[s], (it / kStagesK) & 1, wc, 0x62)) break;
         if (it >= 2 && !mbar_wait(&ctl.tmem_free[tb], ((it >> 1) - 1) & 1, wc, 0x63)) break;
         tc_fence_after();
 #pragma unroll
@@ -658,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ss(tmem + tb * 256, desc_advance(v_k, s * kTileB + offk), desc_advance(ds_k, offk),
                   id_dk, kk != 0);
         }
-        if (!mbar_wait(&ctl.kready[s], (it >> 1) & 1, wc, 0x64)) break;
+        if (!mbar_wait(&ctl.kready[s], (it / kStagesK) & 1, wc, 0x64)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -674,36 +716,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3, c4 = warp >> 2, r = q4 * 32 + lane;
     const int hf = c4 >> 1;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    uint32_t mask0 = 0, mask1 = 0;  // (k > 0) bits of the tile in k stage 0 / 1
+    uint32_t mask[kStagesK] = {0, 0, 0};  // (k > 0) bits of the tile in each k stage
     bool ok = true;
     auto phase_a = [&](int it) {  // k -> k' in place, (k > 0) bits
-      const int s = it & 1;
-      if (!mbar_wait(&ctl.fullK[s], (it >> 1) & 1, wc, 0x65)) {
+      const int s = it % kStagesK;
+      if (!mbar_wait(&ctl.fullK[s], (it / kStagesK) & 1, wc, 0x65)) {
         ok = false;
         return;
       }
       const int n = (tile0 + it) * kRows + r;
       uint32_t m = 0;
       if (n < g.N) {
-        const RowRope rr = row_rope(rs, g, n);
+        const GlobalRowRope rr = global_row_rope(rope, g, b, n);
         quarter_forward_any<NT, NH>(c4, k_st + s * kTileB, r, rr, nullptr, m);
       }
-      if (s) mask1 = m;
-      else mask0 = m;
+#pragma unroll
+      for (int i = 0; i < kStagesK; ++i)  // static register indexing
+        if (i == s) mask[i] = m;
       fence_proxy_async_smem();
       mbar_arrive(&ctl.kready[s]);
     };
     auto phase_b = [&](int it) {  // dk over k', dv over v
-      const int s = it & 1, tb = it & 1;
+      const int s = it % kStagesK, tb = it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&ctl.mma_done[tb], (it >> 1) & 1, wc, 0x66))) {
         ok = false;
         return;
       }
       tc_fence_after();
       const int n = (tile0 + it) * kRows + r;
-      const RowRope rr = row_rope(rs, g, n < g.N ? n : 0);
+      const GlobalRowRope rr = global_row_rope(rope, g, b, n < g.N ? n : 0);
+      uint32_t m = 0;
+#pragma unroll
+      for (int i = 0; i < kStagesK; ++i)
+        if (i == s) m = mask[i];
       quarter_backward_any<NT, NH>(c4, k_st + s * kTileB, r, rr, tmem + lane_base + tb * 256, 1.f,
-                                   ctl.dz, s ? mask1 : mask0, nullptr, nullptr);
+                                   ctl.dz, m, nullptr, nullptr);
       uint8_t* vhalf = v_st + s * kTileB + hf * kHalf;
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
@@ -747,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 constexpr size_t kBwdQSmem = 1024 + 6 * (size_t)kTileB;  // S, q x2, dy x2, g
-constexpr size_t kBwdKSmem = 1024 + 5 * (size_t)kTileB;  // dS, k x2, v x2
+constexpr size_t kBwdKSmem = 1024 + (1 + 2 * kStagesK) * (size_t)kTileB;  // dS, k and v rings
 constexpr size_t kSmemPerBlock = 232448;                  // sm_100 opt-in maximum
 constexpr int kStdNT = 22, kStdNH = 21;
 
@@ -758,7 +805,7 @@ void set_bwd_attrs() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || done[dev]) return;
-  const int q = (int)(kSmemPerBlock - sizeof(BwdQCtl)), k = (int)(kBwdKSmem + kRopeSmemMax);
+  const int q = (int)(kSmemPerBlock - sizeof(BwdQCtl)), k = (int)kBwdKSmem;
   cudaFuncSetAttribute(linattn_bwd_q_kernel<true, kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
   cudaFuncSetAttribute(linattn_bwd_q_kernel<false, kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
   cudaFuncSetAttribute(linattn_bwd_q_kernel<true, -1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
@@ -798,7 +845,7 @@ sana_status linattn_bf16_backward(const sana_shape& s, const LinAttnPlan& plan, 
                 g.T, g.H, g.W);
   set_bwd_attrs();
   const dim3 grid(plan.splits_a, s.heads, s.B);
-  const size_t smq = kBwdQSmem + rope_smem_bytes(g, rope), smk = kBwdKSmem + rope_smem_bytes(g, rope);
+  const size_t smq = kBwdQSmem + rope_smem_bytes(g, rope), smk = kBwdKSmem;
   const bool sd = std_split(rope);
   int* sw = status_word();
   if (gt && sd)
