@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   const int ntiles = (int)((long long)(split + 1) * tiles_total / splits) - tile0;
   const WaitCtx wc{&ctl.abort_flag, status};
   volatile int* abort_flag = &ctl.abort_flag;
+  griddep_launch_next();
 
   if (tid == 0) {
     for (int s = 0; s < kStagesA; ++s) {
@@ -277,25 +278,67 @@ __global__ void __launch_bounds__(kThreadsA, 1)
 // ------------------------------------------------------------------------
 // combine kernel (shared with the fp32 path): fixed-order sum over splits.
 // Grid (batch * heads, slices): each CTA sums one slice of one head's S.
+// Every element is S_prev + p_0 + p_1 + ... in that order; a thread owns four
+// consecutive elements and issues the loads of up to kCombineBatch splits
+// before it adds them, so the reduction is bound by bandwidth, not by the
+// latency of one load after another.
 // ------------------------------------------------------------------------
 constexpr int kCombineSlices = 16;
+constexpr int kCombineBatch = 8;
+
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
 
 __global__ void __launch_bounds__(256)
     linattn_combine_kernel(const float* __restrict__ ws_S, const float* __restrict__ ws_z,
                            int splits, int D, const float* S_prev, const float* z_prev,
                            float* S_state, float* z_state, float* __restrict__ S_f32,
                            float* __restrict__ z_out) {
+  griddep_wait();  // the partials come from the previous launch
+  griddep_launch_next();
   const int bh = blockIdx.x;
   const int DD = D * D;
-  const int per = (DD + (int)gridDim.y - 1) / (int)gridDim.y;
-  const int beg = (int)blockIdx.y * per;
-  const int end = min(DD, beg + per);
   const size_t base = (size_t)bh * DD;
-  for (int idx = beg + threadIdx.x; idx < end; idx += blockDim.x) {
-    float acc = S_prev ? S_prev[base + idx] : 0.f;
-    for (int sp = 0; sp < splits; ++sp) acc += ws_S[((size_t)bh * splits + sp) * DD + idx];
-    if (S_state) S_state[base + idx] = acc;
-    if (S_f32) S_f32[base + idx] = acc;
+  const uintptr_t addr_bits = reinterpret_cast<uintptr_t>(ws_S) |
+                              reinterpret_cast<uintptr_t>(S_prev) |
+                              reinterpret_cast<uintptr_t>(S_state) | reinterpret_cast<uintptr_t>(S_f32);
+  if ((DD & 3) == 0 && (addr_bits & 15u) == 0) {
+    // float4 path: with DD a multiple of 4 and 16-byte aligned buffers every
+    // access is aligned
+    const int DD4 = DD >> 2;
+    const int per = (DD4 + (int)gridDim.y - 1) / (int)gridDim.y;
+    const int beg = (int)blockIdx.y * per;
+    const int end = min(DD4, beg + per);
+    const float4* part = reinterpret_cast<const float4*>(ws_S) + (size_t)bh * splits * DD4;
+    for (int i = beg + threadIdx.x; i < end; i += blockDim.x) {
+      float4 acc = S_prev ? reinterpret_cast<const float4*>(S_prev + base)[i]
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < splits; s0 += kCombineBatch) {
+        float4 p[kCombineBatch];
+#pragma unroll
+        for (int j = 0; j < kCombineBatch; ++j)
+          if (s0 + j < splits) p[j] = part[(size_t)(s0 + j) * DD4 + i];
+#pragma unroll
+        for (int j = 0; j < kCombineBatch; ++j)
+          if (s0 + j < splits) add4(acc, p[j]);
+      }
+      if (S_state) reinterpret_cast<float4*>(S_state + base)[i] = acc;
+      if (S_f32) reinterpret_cast<float4*>(S_f32 + base)[i] = acc;
+    }
+  } else {
+    const int per = (DD + (int)gridDim.y - 1) / (int)gridDim.y;
+    const int beg = (int)blockIdx.y * per;
+    const int end = min(DD, beg + per);
+    for (int idx = beg + threadIdx.x; idx < end; idx += blockDim.x) {
+      float acc = S_prev ? S_prev[base + idx] : 0.f;
+      for (int sp = 0; sp < splits; ++sp) acc += ws_S[((size_t)bh * splits + sp) * DD + idx];
+      if (S_state) S_state[base + idx] = acc;
+      if (S_f32) S_f32[base + idx] = acc;
+    }
   }
   if (blockIdx.y == 0)
     for (int d = threadIdx.x; d < D; d += blockDim.x) {
@@ -311,9 +354,9 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------------
 struct OutSmemCtl {
   uint64_t fullQ[kStagesQ], emptyQ[kStagesQ], qready[kStagesQ];
-  uint64_t fullG[kStagesG], emptyG[kStagesG];
+  uint64_t fullG[kStagesG], ystaged[kStagesG];
   uint64_t mma_done[2], tmem_free[2];
-  uint64_t wsync, hsync[2];  // reusable worker barriers (bounded waits)
+  uint64_t wsync;  // reusable worker barrier (bounded waits)
   uint32_t tmem;
   int abort_flag;
   alignas(16) float den[kStagesQ][4][kRows];
@@ -351,12 +394,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
     for (int s = 0; s < kStagesG; ++s) {
       mbar_init(&ctl.fullG[s], 1);
-      mbar_init(&ctl.emptyG[s], 2);
+      mbar_init(&ctl.ystaged[s], kWorkers);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.mma_done[i], 1);
       mbar_init(&ctl.tmem_free[i], kWorkers);
-      mbar_init(&ctl.hsync[i], kWorkers / 2);
     }
     mbar_init(&ctl.wsync, kWorkers);
     ctl.abort_flag = 0;
@@ -366,6 +408,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     tmem_alloc(&ctl.tmem, 256);
     tmem_relinquish();
   }
+  // everything above overlaps the previous launch's tail; S and z (and Q, G)
+  // are read only after it has finished
+  griddep_wait();
   if (tid < kD) ctl.z[tid] = z_all[(size_t)bh * kD + tid];
   if (tid < kWorkers) {
     // S^T operand: element (e, d) = S[d][e] in bf16, K-major [2 halves of
@@ -405,13 +450,30 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       }
     }
   } else if (warp == kWarpProdG) {
-    // ---------------- G producer (ungated: only hands out the staging buffers)
+    // ---------------- G producer and Y store.  Stage s holds G of a tile, the
+    // workers overwrite it with that tile's Y, this thread stores Y by TMA and
+    // refills the stage once the store has read it (the workers never wait
+    // for a store).  Ungated, the stages only stage Y.
     if (lane == 0) {
       if (kGate) prefetch_tmap(&tm_g);
+      prefetch_tmap(&tm_y);
+      auto store_y = [&](int t) {  // Y of tile t, once all its rows are staged
+        const int st = t % kStagesG;
+        if (!mbar_wait(&ctl.ystaged[st], (t / kStagesG) & 1, wc, 0x22)) return false;
+        uint8_t* src = g_st + st * kTileB;
+        tma_store_3d(&tm_y, src, h * kD, (tile0 + t) * kRows, b);
+        tma_store_3d(&tm_y, src + kHalf, h * kD + 64, (tile0 + t) * kRows, b);
+        bulk_commit();
+        return true;
+      };
+      bool okp = true;
       for (int it = 0; it < ntiles; ++it) {
         const int s = it % kStagesG;
-        if (it >= kStagesG && !mbar_wait(&ctl.emptyG[s], ((it / kStagesG) - 1) & 1, wc, 0x22))
-          break;
+        if (it >= kStagesG) {
+          okp = store_y(it - kStagesG);
+          if (!okp) break;
+          bulk_wait_read0();  // the stage has been read out
+        }
         if (kGate) {
           const int n0 = (tile0 + it) * kRows;
           mbar_arrive_expect_tx(&ctl.fullG[s], kTileB);
@@ -421,6 +483,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           mbar_arrive(&ctl.fullG[s]);
         }
       }
+      for (int t = ntiles > kStagesG ? ntiles - kStagesG : 0; okp && t < ntiles; ++t)
+        okp = store_y(t);
+      bulk_wait0();
     }
   } else if (warp == kWarpMmaB) {
     // ---------------- MMA issuer: D[tok][e] = Q'[tok][d] S[d][e]
@@ -472,7 +537,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       fence_proxy_async_smem();
       mbar_arrive(&ctl.qready[s]);
     };
-    uint32_t n_wsync = 0, n_hsync = 0;
+    uint32_t n_wsync = 0;
     auto epilogue = [&](int it) {
       const int s = it % kStagesQ, tb = it & 1, sg = it % kStagesG;
       bool okw = mbar_wait(&ctl.mma_done[tb], (it >> 1) & 1, wc, 0x27);
@@ -517,15 +582,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
       }
       fence_proxy_async_smem();
-      // the 128 rows of this 64-column half are staged
-      mbar_arrive(&ctl.hsync[hf]);
-      okw = mbar_wait(&ctl.hsync[hf], (n_hsync++) & 1, wc, 0x2a) && okw;
-      if (okw && q4 == 0 && (c4 & 1) == 0 && lane == 0) {
-        tma_store_3d(&tm_y, half, h * kD + hf * 64, (tile0 + it) * kRows, b);
-        bulk_commit();
-        bulk_wait_read0();
-        mbar_arrive(&ctl.emptyG[sg]);
-      }
+      mbar_arrive(&ctl.ystaged[sg]);  // the G producer stores the tile
       ok = okw;
     };
     if (ntiles > 0) prologue(0);
@@ -534,7 +591,6 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       if (!ok) break;
       epilogue(it);
     }
-    if (q4 == 0 && (c4 & 1) == 0 && lane == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -607,8 +663,10 @@ sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, con
                                float* z_state, float* ws_S, float* ws_z, float* S_f32,
                                float* z_out, cudaStream_t st) {
   if (sana_status e = linattn_bf16_partials(s, plan, k, v, rope, g, ws_S, ws_z, st)) return e;
-  linattn_combine_kernel<<<dim3(s.B * s.heads, kCombineSlices), 256, 0, st>>>(
-      ws_S, ws_z, plan.splits_a, kD, S_prev, z_prev, S_state, z_state, S_f32, z_out);
+  const cudaError_t e = launch_dependent(linattn_combine_kernel, dim3(s.B * s.heads, kCombineSlices),
+                                         dim3(256), 0, st, ws_S, ws_z, plan.splits_a, kD, S_prev,
+                                         z_prev, S_state, z_state, S_f32, z_out);
+  if (e != cudaSuccess) return fail(SANA_ERR_CUDA, "linattn_combine_kernel: %s", cudaGetErrorString(e));
   return check_launch("linattn_combine_kernel");
 }
 
@@ -629,18 +687,14 @@ sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, con
   const dim3 grid(plan.splits_b, s.heads, s.B);
   const bool stdsp = is_std_split(rope);
   int* sw = status_word();
-  if (gt && stdsp)
-    linattn_out_kernel<true, kStdNT, kStdNH><<<grid, kThreadsB, smem_b, st>>>(
-        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
-  else if (gt)
-    linattn_out_kernel<true, -1, -1><<<grid, kThreadsB, smem_b, st>>>(
-        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
-  else if (stdsp)
-    linattn_out_kernel<false, kStdNT, kStdNH><<<grid, kThreadsB, smem_b, st>>>(
-        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
-  else
-    linattn_out_kernel<false, -1, -1><<<grid, kThreadsB, smem_b, st>>>(
-        tq, tg, ty, S_f32, z, rope, g, plan.tiles, plan.splits_b, eps, sw);
+  // launched as a programmatic dependent: its prologue overlaps the tail of
+  // the launch that produces S and z
+  auto kern = gt ? (stdsp ? linattn_out_kernel<true, kStdNT, kStdNH> : linattn_out_kernel<true, -1, -1>)
+                 : (stdsp ? linattn_out_kernel<false, kStdNT, kStdNH>
+                          : linattn_out_kernel<false, -1, -1>);
+  const cudaError_t e = launch_dependent(kern, grid, dim3(kThreadsB), smem_b, st, tq, tg, ty, S_f32,
+                                         z, rope, g, plan.tiles, plan.splits_b, eps, sw);
+  if (e != cudaSuccess) return fail(SANA_ERR_CUDA, "linattn_out_kernel: %s", cudaGetErrorString(e));
   return check_launch("linattn_out_kernel");
 }
 
