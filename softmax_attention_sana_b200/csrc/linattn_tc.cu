@@ -28,6 +28,7 @@
 
 #include <cstddef>
 
+#include "pdl.cuh"
 #include "rope_dev.cuh"
 #include "sana_common.cuh"
 #include "sana_internal.h"
@@ -61,6 +62,41 @@ __device__ __forceinline__ float2 pair_cs(const RowRope& rr, int j) {
   return rr.cs(j);
 }
 
+// ---- packed arithmetic: one instruction for two columns
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+// max(x, 0) of both bf16 halves
+__device__ __forceinline__ uint32_t relu_bf2(uint32_t w) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0u));
+  return r;
+}
+// sigmoid of both bf16 halves of w (gate logits) as f32x2, by the tanh
+// identity sigmoid(x) = 1/2 + tanh(x/2)/2 (one MUFU op per value)
+__device__ __forceinline__ uint64_t sigmoid2(uint32_t w) {
+  const float2 g = bf2_to_f2(w);
+  float t0, t1;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(0.5f * g.x));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(0.5f * g.y));
+  return fma2(pk2(t0, t1), pk2(0.5f, 0.5f), pk2(0.5f, 0.5f));
+}
+
 // ReLU + RoPE of one 16-byte chunk (4 rotary pairs starting at pair0) of a
 // swizzled tile row, rewritten in place; the ReLU values are returned.
 template <int NT, int NH>
@@ -70,9 +106,7 @@ __device__ __forceinline__ void relu_rope_chunk(uint8_t* p, const RowRope& rr, i
   uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float2 x = bf2_to_f2(w[i]);
-    x.x = fmaxf(x.x, 0.f);
-    x.y = fmaxf(x.y, 0.f);
+    const float2 x = bf2_to_f2(relu_bf2(w[i]));  // exact: ReLU commutes with widening
     phi_out[2 * i] = x.x;
     phi_out[2 * i + 1] = x.y;
     const float2 r = rotate(x.x, x.y, pair_cs<NT, NH>(rr, pair0 + i));
@@ -99,23 +133,21 @@ template <int NT, int NH, int C4>
 __device__ __forceinline__ float quarter_query(uint8_t* tile, int r, const RowRope& rr,
                                                const float* z) {
   uint8_t* half = tile + (C4 >> 1) * kHalf;
-  float den = 0.f;
+  uint64_t den2 = pk2(0.f, 0.f);  // even and odd columns, summed at the end
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     float ph[8];
     relu_rope_chunk<NT, NH>(half + sw128_off(r, (C4 & 1) * 4 + ch), rr, C4 * 16 + ch * 4, ph);
     const float4 z0 = *reinterpret_cast<const float4*>(z + C4 * 32 + ch * 8);
     const float4 z1 = *reinterpret_cast<const float4*>(z + C4 * 32 + ch * 8 + 4);
-    den = fmaf(ph[0], z0.x, den);
-    den = fmaf(ph[1], z0.y, den);
-    den = fmaf(ph[2], z0.z, den);
-    den = fmaf(ph[3], z0.w, den);
-    den = fmaf(ph[4], z1.x, den);
-    den = fmaf(ph[5], z1.y, den);
-    den = fmaf(ph[6], z1.z, den);
-    den = fmaf(ph[7], z1.w, den);
+    den2 = fma2(pk2(ph[0], ph[1]), pk2(z0.x, z0.y), den2);
+    den2 = fma2(pk2(ph[2], ph[3]), pk2(z0.z, z0.w), den2);
+    den2 = fma2(pk2(ph[4], ph[5]), pk2(z1.x, z1.y), den2);
+    den2 = fma2(pk2(ph[6], ph[7]), pk2(z1.z, z1.w), den2);
   }
-  return den;
+  float d0, d1;
+  up2(den2, d0, d1);
+  return d0 + d1;
 }
 
 // ------------------------------------------------------------------------
@@ -547,6 +579,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       okw = __all_sync(0xffffffffu, okw);  // tcgen05.ld is warp-collective
       const float inv =
           1.f / (ctl.den[s][0][r] + ctl.den[s][1][r] + ctl.den[s][2][r] + ctl.den[s][3][r] + eps);
+      const uint64_t inv2 = pk2(inv, inv);
       uint32_t acc[32];
       if (okw) {
         tc_fence_after();
@@ -569,13 +602,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           uint32_t out[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            float y0 = __uint_as_float(acc[ch * 8 + 2 * i]) * inv;
-            float y1 = __uint_as_float(acc[ch * 8 + 2 * i + 1]) * inv;
-            if (kGate) {
-              const float2 gg = bf2_to_f2(gw[i]);
-              y0 *= sigmoid_fast(gg.x);
-              y1 *= sigmoid_fast(gg.y);
-            }
+            uint64_t y2 = mul2(pk2(__uint_as_float(acc[ch * 8 + 2 * i]),
+                                   __uint_as_float(acc[ch * 8 + 2 * i + 1])),
+                               inv2);
+            if (kGate) y2 = mul2(y2, sigmoid2(gw[i]));
+            float y0, y1;
+            up2(y2, y0, y1);
             out[i] = f2_to_bf2(y0, y1);
           }
           *p = make_uint4(out[0], out[1], out[2], out[3]);
