@@ -49,6 +49,12 @@ Readings where the pages are silent:
   print no backward; linattn_backward is the chain rule through the forward
   as written (ReLU derivative 1 for x > 0, 0 otherwise), pinned by finite
   differences.
+* MX formats ([SV2] Experiments name MXFP4 weights and MXFP8 activations
+  for the linear GEMMs): the OCP Microscaling v1.0 definitions.
+  - Blocks are 32 elements along the contraction axis, with one E8M0
+    exponent s = floor(log2 amax) - emax_elem.
+  - Elements are E4M3 (max 448) or E2M1 (max 6), rounded to nearest-even
+    and saturated.
 * Sparse anchor ([SV2] Experiments and [SV2-abs] say only that the
   deployment stack applies sparse attention to the softmax anchors): queries
   in blocks of 256 tokens, keys in tiles of 128; each block keeps the `keep`
@@ -578,6 +584,95 @@ def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
             partial = None
     h, _ = attnres_route(sources(), w_attn, rms_eps)
     return h
+
+
+# --------------------------------------------------------------------------
+# MX block-scaled formats for the projection GEMMs  ([SV2] Experiments:
+# low-precision inference quantises only the linear GEMM layers, weights to
+# MXFP4 and activations to MXFP8; attention stays bf16)
+# --------------------------------------------------------------------------
+
+# The pages name the formats without defining them.  Reading: the OCP
+# Microscaling (MX) v1.0 definitions.  A block of 32 consecutive elements
+# along the contraction axis shares one scale 2^s (an E8M0 exponent,
+# s in [-127, 127]).  Each element is an FP8 E4M3 value (MXFP8) or an FP4 E2M1
+# value (MXFP4).
+E4M3 = {"name": "e4m3", "mbits": 3, "bias": 7, "emax": 8, "maxval": 448.0}
+E2M1 = {"name": "e2m1", "mbits": 1, "bias": 1, "emax": 2, "maxval": 6.0}
+MX_BLOCK = 32
+MX_SCALE_MIN, MX_SCALE_MAX = -127, 127
+
+
+def fp_values(fmt):
+    """The non-negative finite values of an element format, in code order.
+
+    Subnormals are m * 2^(1 - bias - mbits), for m < 2^mbits. Normals are
+    (1 + m / 2^mbits) * 2^(e - bias), for biased exponents e >= 1. The list
+    stops at the format's largest finite value."""
+    mb, bias = fmt["mbits"], fmt["bias"]
+    vals = [m * 2.0 ** (1 - bias - mb) for m in range(2 ** mb)]
+    e = 1
+    while True:
+        for m in range(2 ** mb):
+            v = (1 + m / 2 ** mb) * 2.0 ** (e - bias)
+            if v > fmt["maxval"]:
+                return np.array(vals)
+            vals.append(v)
+        e += 1
+
+
+def round_to_format(x, fmt):
+    """Round to the nearest value of the element format.
+
+    Ties go to the even code, and a magnitude above the largest finite value
+    saturates to it. Consecutive non-negative values have consecutive codes,
+    so an even index in fp_values is an even code."""
+    x = np.asarray(x, np.float64)
+    vals = fp_values(fmt)
+    a = np.minimum(np.abs(x), fmt["maxval"])
+    i = np.clip(np.searchsorted(vals, a), 1, len(vals) - 1)  # vals[i-1] < a <= vals[i]
+    lo, hi = vals[i - 1], vals[i]
+    up = (a - lo > hi - a) | ((a - lo == hi - a) & (i % 2 == 0))
+    return np.sign(x) * np.where(up, hi, lo)
+
+
+def mx_quantize(x, fmt, block=MX_BLOCK):
+    """MX quantisation along the last axis, which is the contraction axis.
+
+    Each block of `block` elements gets the exponent
+    s = floor(log2(max |x|)) - emax(fmt), clamped to the E8M0 range. An
+    all-zero block takes the smallest exponent. The elements are x / 2^s,
+    rounded by round_to_format. Returns (elements, s), with s of shape
+    x.shape[:-1] + (K / block,)."""
+    x = np.asarray(x, np.float64)
+    K = x.shape[-1]
+    assert K % block == 0, "the contraction length must be a multiple of the block"
+    xb = x.reshape(*x.shape[:-1], K // block, block)
+    amax = np.max(np.abs(xb), axis=-1)
+    _, ex = np.frexp(amax)  # amax = f * 2^ex with f in [1/2, 1): floor(log2 amax) = ex - 1
+    s = np.where(amax > 0, ex - 1 - fmt["emax"], MX_SCALE_MIN)
+    s = np.clip(s, MX_SCALE_MIN, MX_SCALE_MAX).astype(np.int64)
+    el = round_to_format(xb / np.exp2(s)[..., None], fmt)
+    return el.reshape(x.shape), s
+
+
+def mx_dequantize(el, s, block=MX_BLOCK):
+    """Elements times their block's scale."""
+    el = np.asarray(el, np.float64)
+    K = el.shape[-1]
+    eb = el.reshape(*el.shape[:-1], K // block, block)
+    return (eb * np.exp2(s)[..., None]).reshape(el.shape)
+
+
+def mx_linear(x, w, block=MX_BLOCK):
+    """The quantised projection y = Q8(x) Q4(w)^T.
+
+    Activations x (M, K) are MXFP8 (E4M3 elements). Weights w (N, K) are
+    MXFP4 (E2M1 elements). Both are blocked along K, and the dequantised
+    operands are multiplied in float64."""
+    xq = mx_dequantize(*mx_quantize(x, E4M3, block), block)
+    wq = mx_dequantize(*mx_quantize(w, E2M1, block), block)
+    return xq @ wq.T
 
 
 # --------------------------------------------------------------------------

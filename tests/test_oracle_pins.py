@@ -601,3 +601,119 @@ def test_stack_without_attnres_is_residual_composition():
             a = orc.linattn_bruteforce(q, k, v, grid, split, heads, gate=g)
         ref = ref + a @ ws[l]["o"].T
     assert rel(out, ref) < 1e-12
+
+
+# ---------------------------------------------------------------- MX formats (projection GEMMs)
+
+def _decode_e4m3(code):
+    """Value of an 8-bit E4M3 code from its fields (None for the NaN codes)."""
+    sign, e, m = code >> 7, (code >> 3) & 15, code & 7
+    if e == 15 and m == 7:
+        return None
+    mag = m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+    return -mag if sign else mag
+
+
+def _decode_e2m1(code):
+    sign, e, m = code >> 3, (code >> 1) & 3, code & 1
+    mag = m * 0.5 if e == 0 else (1 + m / 2) * 2.0 ** (e - 1)
+    return -mag if sign else mag
+
+
+def test_mx_element_grids_match_the_bit_layouts_and_torch():
+    e4 = sorted({v for c in range(256) if (v := _decode_e4m3(c)) is not None and v >= 0})
+    assert np.array_equal(orc.fp_values(orc.E4M3), np.array(e4))
+    # torch's float8_e4m3fn, read code by code
+    t = torch.arange(128, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(orc.fp_values(orc.E4M3), t[:127]) and np.isnan(t[127])
+    e2 = sorted({_decode_e2m1(c) for c in range(16) if _decode_e2m1(c) >= 0})
+    assert np.array_equal(orc.fp_values(orc.E2M1), np.array(e2))
+    assert orc.fp_values(orc.E2M1).tolist() == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+
+def test_mx_rounding_matches_torch_float8_including_ties():
+    g = np.random.default_rng(7)
+    vals = orc.fp_values(orc.E4M3)
+    mids = (vals[1:] + vals[:-1]) / 2  # exact ties, representable in float32
+    x = np.concatenate([mids, -mids, g.uniform(-448, 448, 4000),
+                        g.standard_normal(2000) * 2.0 ** g.integers(-12, 8, 2000)])
+    x = np.clip(x, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(orc.round_to_format(x.astype(np.float64), orc.E4M3), ref)
+
+
+def test_mx_round_e2m1_hand_worked():
+    x = [0.2, 0.25, 0.3, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 5.5, 7.0, -2.5, -0.25]
+    # ties go to the even code: 0.25 -> 0, 0.75 -> 1, 1.25 -> 1, 1.75 -> 2,
+    # 2.5 -> 2, 3.5 -> 4, 5 -> 4; above 6 saturates
+    exp = [0.0, 0.0, 0.5, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0, 6.0, -2.0, -0.0]
+    assert orc.round_to_format(x, orc.E2M1).tolist() == exp
+
+
+def test_mx_scale_rule_and_saturation():
+    x = np.zeros((1, 32))
+    x[0, :4] = [500.0, 1.0, -2.0, 3.0]
+    el, s = orc.mx_quantize(x, orc.E4M3)
+    # floor(log2 500) = 8 = emax: scale 2^0; 500 saturates to 448
+    assert s.tolist() == [[0]] and el[0, :4].tolist() == [448.0, 1.0, -2.0, 3.0]
+    el, s = orc.mx_quantize(x, orc.E2M1)
+    # floor(log2 500) - 2 = 6: 500 / 64 = 7.8 -> 6, 1/64 -> 0, 3/64 -> 0
+    assert s.tolist() == [[6]] and el[0, :4].tolist() == [6.0, 0.0, -0.0, 0.0]
+    z, sz = orc.mx_quantize(np.zeros((2, 64)), orc.E4M3)
+    assert not z.any() and (sz == orc.MX_SCALE_MIN).all()
+
+
+def test_mx_quantize_is_invariant_under_power_of_two_scaling():
+    x = rand(6, 96)
+    for fmt in (orc.E4M3, orc.E2M1):
+        el, s = orc.mx_quantize(x, fmt)
+        for j in (-20, -3, 5, 31):
+            el2, s2 = orc.mx_quantize(x * 2.0 ** j, fmt)
+            assert np.array_equal(el2, el) and np.array_equal(s2, s + j)
+
+
+def test_mx_representable_blocks_round_trip_exactly():
+    g = np.random.default_rng(11)
+    for fmt in (orc.E4M3, orc.E2M1):
+        vals = orc.fp_values(fmt)
+        top = vals[vals >= 2.0 ** fmt["emax"]]  # the block max lies in the top binade
+        el = g.choice(vals, size=(5, 64)) * g.choice([-1.0, 1.0], size=(5, 64))
+        el[:, 0], el[:, 32] = g.choice(top, 5), -g.choice(top, 5)
+        s = g.integers(-10, 10, size=(5, 2))
+        x = orc.mx_dequantize(el, s)
+        el2, s2 = orc.mx_quantize(x, fmt)
+        assert np.array_equal(s2, s) and np.array_equal(el2, el)
+
+
+def test_mx_quantize_error_within_half_an_ulp_or_saturation():
+    x = rand(8, 128) * np.exp(rand(8, 128))
+    for fmt in (orc.E4M3, orc.E2M1):
+        el, s = orc.mx_quantize(x, fmt)
+        deq = orc.mx_dequantize(el, s)
+        scale = np.repeat(np.exp2(s), 32, axis=-1)
+        u = np.abs(x) / scale  # magnitude in element units
+        half_ulp = np.exp2(np.floor(np.log2(np.maximum(u, 2.0 ** (1 - fmt["bias"])))) - fmt["mbits"] - 1)
+        sat = u > fmt["maxval"]
+        err = np.abs(deq - x) / scale
+        assert (err[~sat] <= half_ulp[~sat] * (1 + 1e-12)).all()
+        assert np.allclose(err[sat], u[sat] - fmt["maxval"], rtol=0, atol=1e-12)
+        assert (u < 2.0 ** (fmt["emax"] + 1)).all()  # the scale rule bounds every block
+
+
+def test_mx_linear_is_the_product_of_the_dequantised_operands():
+    g = np.random.default_rng(5)
+    M, N, K = 7, 5, 96
+    xe = g.choice(orc.fp_values(orc.E4M3), (M, K)) * g.choice([-1, 1], (M, K))
+    we = g.choice(orc.fp_values(orc.E2M1), (N, K)) * g.choice([-1, 1], (N, K))
+    xe[:, ::32], we[:, ::32] = 448.0, 6.0  # block maxima in the top binade
+    x = orc.mx_dequantize(xe, g.integers(-4, 4, (M, K // 32)))
+    w = orc.mx_dequantize(we, g.integers(-4, 4, (N, K // 32)))
+    # exactly representable operands: the quantised GEMM is the plain product
+    assert np.array_equal(orc.mx_linear(x, w), x @ w.T)
+    # and on general operands it differs from the plain product by the
+    # rounding of each operand only
+    a, b = rand(M, K), rand(N, K)
+    qa = orc.mx_dequantize(*orc.mx_quantize(a, orc.E4M3))
+    qb = orc.mx_dequantize(*orc.mx_quantize(b, orc.E2M1))
+    assert np.allclose(orc.mx_linear(a, b), qa @ qb.T, rtol=0, atol=1e-12)
+    assert rel(orc.mx_linear(a, b), a @ b.T) < 0.5
