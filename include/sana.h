@@ -340,9 +340,15 @@ SANA_API sana_status sana_hybrid_stack_fwd(const sana_shape* shape, const sana_s
  * sana_linattn_noalloc_scratch_bytes() bytes (16 MiB) held on every GPU that
  * loads the library until the process exits.  Shapes needing more scratch
  * than that (sana_linattn_workspace_size() larger) return
- * SANA_ERR_UNSUPPORTED.  All calls share the array: calls that overlap on the
- * GPU (different streams or host threads) race.  The first call on a device
- * looks up the array's device address; make it before any stream capture.
+ * SANA_ERR_UNSUPPORTED; for bf16 at head_dim 128 that is B * heads >= 128.
+ * All calls share the array: calls that overlap on the GPU (different streams
+ * or host threads) race.  The first call on a device (and the first after a
+ * device reset) looks up the array's device address; make it before any
+ * stream capture.  Under lazy module loading (the CUDA 12 default) the
+ * library's device code, and the array with it, is loaded onto a device by
+ * the first library call made there, which may synchronise the device: make
+ * one call (or call sana_linattn_noalloc_scratch_bytes() after any other
+ * library call on that device) at initialisation time.
  * ------------------------------------------------------------------------- */
 SANA_API size_t sana_linattn_noalloc_scratch_bytes(void);
 SANA_API sana_status sana_linattn_fwd_noalloc(const sana_shape* shape, sana_dtype dtype,

@@ -13,9 +13,16 @@
 // library and stays resident until the process exits.  Every call shares it,
 // so calls whose kernels overlap on the GPU (other streams, other host
 // threads) race on it.  The kernels fully overwrite the parts they read, so
-// nothing needs clearing between calls.  The first call on a device looks up
-// the array's device address (cudaGetSymbolAddress); make that first call
-// before any stream capture.
+// nothing needs clearing between calls.  The first call on a device (and the
+// first after a device reset) looks up the array's device address with
+// cudaGetSymbolAddress; make that first call before any stream capture.
+//
+// Under lazy module loading (the CUDA 12 default) the library's device code,
+// and with it this array, is loaded onto a device by the first library call
+// made there, and that load may synchronise the device.  Callers for whom this
+// matters should make one call at initialisation time.
+#include <mutex>
+
 #include "sana_common.cuh"
 #include "sana_internal.h"
 
@@ -25,17 +32,27 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the array on the current device, looked up once per
-// device.  In host code the array's name is only a host-side stand-in, so the
-// address must come from cudaGetSymbolAddress with that device current.
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address must come from
+// cudaGetSymbolAddress with that device current.  It is looked up once per
+// device and context: after a device reset the device gets a new context in
+// which the array may sit elsewhere, and a changed context id forces a new
+// lookup.  The mutex makes first calls from several host threads safe.
 void* scratch_ptr(sana_status* st) {
-  static void* addr[64] = {nullptr};
+  struct Slot {
+    unsigned long long ctx;
+    void* addr;
+  };
+  static Slot slots[64] = {};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     *st = fail(SANA_ERR_CUDA, "sana_linattn_fwd_noalloc: no current device");
     return nullptr;
   }
-  if (!addr[dev]) {
+  std::lock_guard<std::mutex> lock(mu);
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0 || slots[dev].ctx != ctx || !slots[dev].addr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) {
@@ -43,10 +60,11 @@ void* scratch_ptr(sana_status* st) {
                  cudaGetErrorString(e));
       return nullptr;
     }
-    addr[dev] = p;
+    // the lookup makes the primary context current when none was
+    slots[dev] = Slot{current_context_id(), p};
   }
   *st = SANA_OK;
-  return addr[dev];
+  return slots[dev].addr;
 }
 
 }  // namespace

@@ -38,16 +38,50 @@ sana_status check_launch(const char* what) {
   return SANA_OK;
 }
 
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 int* status_word() {
-  static int* addr[64] = {nullptr};
+  // One slot per device, valid for the context it was looked up in: a device
+  // reset gives the device a new context whose copy of the word may sit at a
+  // new address, so a changed context id forces a new lookup.
+  struct Slot {
+    unsigned long long ctx;
+    int* addr;
+  };
+  static Slot slots[64] = {};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int*>(p);
-  }
-  return addr[dev];
+  std::lock_guard<std::mutex> lock(mu);
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0 && slots[dev].ctx == ctx && slots[dev].addr) return slots[dev].addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+  // the lookup makes the primary context current when none was
+  slots[dev] = Slot{current_context_id(), static_cast<int*>(p)};
+  return slots[dev].addr;
 }
 
 // ---------------------------------------------------------------- failure-detection self-test

@@ -19,6 +19,9 @@ constexpr int kNumSMs = 148;
 
 sana_status fail(sana_status st, const char* fmt, ...);
 sana_status check_launch(const char* what);
+// Unique id of the calling thread's current CUDA context (cuCtxGetId), 0 if
+// there is none yet or the driver does not provide it.
+unsigned long long current_context_id();
 // Device address of the status word of the current device.
 int* status_word();
 

@@ -603,6 +603,53 @@ def test_stack_without_attnres_is_residual_composition():
     assert rel(out, ref) < 1e-12
 
 
+# Textbook values of the logistic function: sigma(1), sigma(2).
+SIGMA_1 = 0.7310585786300049
+SIGMA_2 = 0.8807970779778823
+
+
+def test_silu_closed_form_values_and_odd_part():
+    """SiLU(x) = x sigma(x): SiLU(0) = 0, SiLU(1) = sigma(1), SiLU(-1) =
+    -(1 - sigma(1)), SiLU(2) = 2 sigma(2), SiLU(-2) = -2 (1 - sigma(2)); and
+    SiLU(x) - SiLU(-x) = x for every x (sigma(x) + sigma(-x) = 1), which
+    x * sigma(-x) or a missing factor of x would break."""
+    got = orc.silu(np.array([0.0, 1.0, -1.0, 2.0, -2.0]))
+    exp = np.array([0.0, SIGMA_1, -(1 - SIGMA_1), 2 * SIGMA_2, -2 * (1 - SIGMA_2)])
+    np.testing.assert_allclose(got, exp, rtol=1e-15, atol=1e-16)
+    x = rand(50) * 5
+    np.testing.assert_allclose(orc.silu(x) - orc.silu(-x), x, rtol=1e-13, atol=1e-14)
+    assert orc.silu(np.array([60.0]))[0] == pytest.approx(60.0, rel=1e-15)
+    assert abs(orc.silu(np.array([-60.0]))[0]) < 1e-24
+
+
+def test_ffn_sublayer_hand_worked():
+    """C = 2, hidden 3, asymmetric weights (a transposed W_up or W_down fails):
+    x = (1, -2); W_up rows (1, 0), (0, 1), (1, 1) give pre-activations
+    (1, -2, -1); u = SiLU of them = (sigma(1), -2 (1 - sigma(2)), -(1 - sigma(1)));
+    W_down rows (1, 2, 3), (0, -1, 1) give (u0 + 2 u1 + 3 u2, u2 - u1)."""
+    xh = np.array([[1.0, -2.0]])
+    Wl = dict(up=np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]]),
+              down=np.array([[1.0, 2.0, 3.0], [0.0, -1.0, 1.0]]))
+    u0, u1, u2 = SIGMA_1, -2 * (1 - SIGMA_2), -(1 - SIGMA_1)
+    exp = np.array([[u0 + 2 * u1 + 3 * u2, u2 - u1]])
+    np.testing.assert_allclose(orc._ffn_sublayer(xh, Wl), exp, rtol=1e-14)
+
+
+def test_stack_ffn_sublayer_enters_the_residual_stream():
+    """One layer without AttnRes, W_o = 0, FFN on: x' = x + FFN(RMSNorm x).
+    x = (2, -4, 2, -4) has mean square 10, so RMSNorm x = x / sqrt(10 + eps);
+    with W_up = I and W_down = 2 I the output is x + 2 SiLU(x / sqrt(10 + eps))."""
+    grid, split, heads, D = (1, 1, 1), (0, 0, 1), 2, 2
+    C = heads * D
+    x = np.array([[[2.0, -4.0, 2.0, -4.0]]])
+    ws = [dict(qkvg=rand(4 * C, C), o=np.zeros((C, C)), up=np.eye(C), down=2 * np.eye(C))]
+    out = orc.hybrid_stack(x, ws, None, None, grid, split, heads, 1, use_attnres=False, ffn=True)
+    r = math.sqrt(10 + orc.RMS_EPS)
+    xn = x / r
+    exp = x + 2 * xn / (1 + np.exp(-xn))
+    np.testing.assert_allclose(out, exp, rtol=1e-14)
+
+
 # ---------------------------------------------------------------- MX formats (projection GEMMs)
 
 def _decode_e4m3(code):
