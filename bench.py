@@ -42,12 +42,27 @@ LAYER_FLOPS = 4 * WL.B * WL.N * WL.heads * WL.D ** 2   # K'^T V and Q' S
 FALLBACK_HBM_GBS = 6650.0
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
         return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 tensor peak (burst: the anchor is timed on its own)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        if "bf16_tflops" in d:
+            return d["bf16_tflops"], "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash():
@@ -217,16 +232,21 @@ def run_reference(args, world, rank):
     n_tok = int(min(WL.N, max(512, budget / per_tok)))
     for _ in range(args.warmup):
         oracle_sample(1, n_tok)
-    vals = []
+    vals, secs = [], []
     desc = ""
     for _ in range(args.steps):
-        v, _, desc = oracle_sample(1, n_tok)
+        v, dt, desc = oracle_sample(1, n_tok)
         vals.append(v)
+        secs.append(dt)
     value = float(np.median(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * WL.B * WL.N / value, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * float(np.median(secs)),
+        "ms_per_step_kind": "measured: wall time of one step's bounded sample (1 head x "
+                            f"{n_tok} tokens); value is that sample's rate scaled to a whole layer",
+        "extrapolated_ms_per_layer": 1e3 * WL.B * WL.N / value,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
@@ -341,23 +361,80 @@ def components(sana, args):
         f()
     ms = time_loop(f, 10)
     out["gemm_qkvg_720p"] = {"ms": ms, "TFLOP_per_s": 2 * WL.N * 4 * WL.C * WL.C / (ms / 1e3) / 1e12}
+    bf16_ms = ms
+    # the same projection quantised: MXFP4 weights (quantised once, untimed),
+    # MXFP8 activations quantised on the fly (sana_mx_linear), and the
+    # block-scaled GEMM alone on pre-quantised activations
+    try:
+        wq, wsc = sana.mx_quantize(Wq, fp4=True)
+        xq, xs = sana.mx_quantize(A)
+        ws_mx = torch.empty(sana._lib.lib.sana_mx_linear_workspace_size(WL.N, WL.C),
+                            dtype=torch.uint8, device="cuda")
+        f = lambda: sana.mx_linear(A, wq, wsc, 4 * WL.C, out=Yq, ws=ws_mx)
+        for _ in range(3):
+            f()
+        ms = time_loop(f, 10)
+        g = lambda: sana.mx_gemm(xq, xs, wq, wsc, 4 * WL.C, out=Yq)
+        for _ in range(3):
+            g()
+        ms_g = time_loop(g, 10)
+        q = lambda: sana.mx_quantize(A)
+        ms_q = time_loop(q, 10)
+        flops = 2 * WL.N * 4 * WL.C * WL.C
+        out["mx_linear_qkvg_720p"] = {
+            "ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12, "vs_bf16_gemm": bf16_ms / ms,
+            "gemm_ms": ms_g, "gemm_TFLOP_per_s": flops / (ms_g / 1e3) / 1e12,
+            "frac_of_nominal_fp8_peak": flops / (ms_g / 1e3) / 1e12 / (2 * SPEC_BF16_TFLOPS),
+            "activation_quantise_ms": ms_q,
+            "activation_quantise_GB_per_s": (WL.N * WL.C * 3 + WL.N * WL.C / 32) / (ms_q / 1e3) / 1e9}
+        del wq, wsc, xq, xs, ws_mx
+    except Exception as e:  # keep the rest of the line if this row fails
+        out["mx_linear_qkvg_720p"] = {"unavailable": str(e)[:200]}
     del A, Wq, Yq
     # softmax anchor at 720p/5s
     if args.no_anchor:
         out["softmax_anchor_720p"] = {"skipped": "--no-anchor"}
         return out
     try:
+        grid = (WL.T, WL.H, WL.W)
         q, k, v, g = (t.cuda() for t in si.qkvg(WL))
         rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
         ws = torch.empty(int(4 * TENSOR_BYTES // 2 + (1 << 20)), dtype=torch.uint8, device="cuda")
         y = torch.empty_like(q)
-        f = lambda: sana.softmax_anchor_fwd(q, k, v, g, rope, (WL.T, WL.H, WL.W), WL.heads, out=y,
-                                            ws=ws)
+        flops = 4 * WL.N * WL.N * WL.heads * WL.D
+        # phase 1: the RoPE prepass (Q and K rotated, Q scaled by scale * log2 e)
+        qr, kr = torch.empty_like(q), torch.empty_like(k)
+        mul = WL.D ** -0.5 * 1.4426950408889634
+        pre = lambda: (sana.rope_apply(q, rope, grid, WL.heads, mul=mul, out=qr),
+                       sana.rope_apply(k, rope, grid, WL.heads, out=kr))
+        for _ in range(3):
+            pre()
+        ms_pre = time_loop(pre, 20)
+        out["anchor_rope_prepass_720p"] = {
+            "ms": ms_pre, "launches": 2, "GB_per_s": 4 * TENSOR_BYTES / (ms_pre / 1e3) / 1e9,
+            "frac_of_hbm_peak": 4 * TENSOR_BYTES / (ms_pre / 1e3) / 1e9 / peaks()[0],
+            "algorithmic_bytes": 4 * TENSOR_BYTES, "l2": "no flush: 4 x 464.5 MB per call"}
+        # phase 2: the attention kernel alone on the rotated operands
+        att = lambda: sana.softmax_anchor_rotated_fwd(qr, kr, v, g, grid, WL.heads, out=y)
+        att()
+        ms_att = time_loop(att, 3)
+        tp, tp_kind = tensor_peak()
+        ach = flops / (ms_att / 1e3) / 1e12
+        out["anchor_kernel_720p"] = {"ms": ms_att, "TFLOP_per_s": ach}
+        anchor_roof = {"bound": "tensor", "kernel": "anchor_kernel (QK^T, softmax, PV; 720p/5s)",
+                       "achieved": ach, "peak": tp, "unit": "TFLOP/s", "frac": ach / tp,
+                       "peak_kind": tp_kind + " burst (cuBLAS bf16)", "spec_peak": SPEC_BF16_TFLOPS,
+                       "spec_frac": ach / SPEC_BF16_TFLOPS, "traffic": None,
+                       "algorithmic_flops_per_launch": flops, "ms_per_launch": ms_att}
+        out["_anchor_roofline"] = anchor_roof
+        # the whole call (prepass + kernel)
+        f = lambda: sana.softmax_anchor_fwd(q, k, v, g, rope, grid, WL.heads, out=y, ws=ws)
         f()
         ms = time_loop(f, 3)
-        flops = 4 * WL.N * WL.N * WL.heads * WL.D
-        out["softmax_anchor_720p"] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}
+        out["softmax_anchor_720p"] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12,
+                                      "frac_of_spec_roofline": (flops / SPEC_BF16_TFLOPS / 1e12 * 1e3) / ms}
         dense_ms = ms
+        del qr, kr
         # block-sparse anchor: each 256-query block keeps a quarter of the 591
         # key tiles (selection by pooled logits included in the timing)
         nkt = sana.anchor_tile_count(WL.N)
@@ -379,17 +456,27 @@ def components(sana, args):
     except Exception as e:  # not built yet
         out["softmax_anchor_720p"] = {"unavailable": str(e)[:200]}
     # whole stacks on the 720p/5s grid: the 4-layer 3:1 group (no AttnRes, no
-    # FFN) and the 16-layer AttnRes stack with FFN 3C
-    if args.stacks:
+    # FFN), the same with block-sparse anchors, and the 16-layer AttnRes stack
+    # with FFN 3C (weights drawn on the device, N(0, 1/fan_in))
+    if not args.no_stacks:
         grid = (WL.T, WL.H, WL.W)
         rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
         keep = (sana.anchor_tile_count(WL.N) + 3) // 4
         for name, layers, attnres, ffn, kt in (("stack_720p_group4", 4, False, 0, 0),
                                                 ("stack_720p_group4_sparse25", 4, False, 0, keep),
                                                 ("stack_720p_attnres16", 16, True, 3, 0)):
-            x = si.normal(5000 + layers, (1, WL.N, WL.C)).cuda()
-            ws_l = [{k2: t.cuda() for k2, t in d.items()}
-                    for d in si.projection_weights(5, layers, WL.C, ffn)]
+            gen = torch.Generator(device="cuda")
+            gen.manual_seed(5000 + layers)
+            rn = lambda *sh, sc=1.0: (torch.randn(sh, generator=gen, device="cuda") * sc).to(
+                torch.bfloat16)
+            x = rn(1, WL.N, WL.C)
+            C, F = WL.C, ffn * WL.C
+            ws_l = []
+            for _ in range(layers):
+                d = {"qkvg": rn(4 * C, C, sc=C ** -0.5), "o": rn(C, C, sc=C ** -0.5)}
+                if ffn:
+                    d["up"], d["down"] = rn(F, C, sc=C ** -0.5), rn(C, F, sc=F ** -0.5)
+                ws_l.append(d)
             w_attn, w_ffn = (t.cuda() for t in si.router_queries(5, WL.C))
             cfg = sana.stack_config(layers, block_span=8, use_attnres=attnres, ffn_mult=ffn,
                                     anchor_keep_tiles=kt)
@@ -404,8 +491,12 @@ def components(sana, args):
             if kt:  # executed anchor work of the kept tiles
                 nan = 4 * WL.N * min(WL.N, kt * 128) * WL.heads * WL.D
             flops = nanc * nan + (layers - nanc) * lin + layers * proj
+            tp, tp_kind = tensor_peak()
             out[name] = {"ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12, "layers": layers,
-                         "attnres": attnres, "ffn_mult": ffn}
+                         "attnres": attnres, "ffn_mult": ffn, "flops": flops,
+                         "frac_of_tensor_peak": flops / (ms / 1e3) / 1e12 / tp,
+                         "frac_of_spec_tensor_peak": flops / (ms / 1e3) / 1e12 / SPEC_BF16_TFLOPS,
+                         "timing": "2 calls after 1 warm-up, CUDA events"}
             if kt:
                 out[name]["anchor_keep_tiles"] = kt
             del x, ws_l, y
@@ -541,6 +632,9 @@ def run_ours(args, world, rank, local):
         "cpu_baseline": cpu,
     }
     if comp is not None:
+        anchor_roof = comp.pop("_anchor_roofline", None)
+        if anchor_roof is not None:
+            line["anchor_roofline"] = anchor_roof
         line["components"] = comp
     print(json.dumps(line), flush=True)
 
@@ -680,6 +774,26 @@ def run_sparse_only(args):
                       "TFLOP_per_s_executed": kept / (ms / 1e3) / 1e12}), flush=True)
 
 
+def run_mx_only(args):
+    """The MX projection of the 720p QKVG shape (75,600 x 3072 activations
+    quantised on the fly against 12,288 x 3072 MXFP4 weights): K steps."""
+    import softmax_attention_sana_b200 as sana
+    A = torch.randn(WL.N, WL.C, device="cuda", dtype=torch.bfloat16)
+    W = torch.randn(4 * WL.C, WL.C, device="cuda", dtype=torch.bfloat16) * WL.C ** -0.5
+    Y = torch.empty(WL.N, 4 * WL.C, device="cuda", dtype=torch.bfloat16)
+    wq, wsc = sana.mx_quantize(W, fp4=True)
+    ws = torch.empty(sana._lib.lib.sana_mx_linear_workspace_size(WL.N, WL.C), dtype=torch.uint8,
+                     device="cuda")
+    f = lambda: sana.mx_linear(A, wq, wsc, 4 * WL.C, out=Y, ws=ws)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    flops = 2 * WL.N * 4 * WL.C * WL.C
+    print(json.dumps({"mx_linear_qkvg_720p_ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -694,8 +808,8 @@ def main():
                     help="seconds the --impl reference run aims to take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-anchor", action="store_true", help="leave the anchor out of the components")
-    ap.add_argument("--stacks", action="store_true",
-                    help="also time the 4-layer group and the 16-layer AttnRes stack")
+    ap.add_argument("--no-stacks", action="store_true",
+                    help="leave the 4-layer group and the 16-layer AttnRes stack out of the components")
     ap.add_argument("--anchor-only", action="store_true",
                     help="run only the 480p-shaped softmax anchor (a small case for profiling)")
     ap.add_argument("--scan-only", action="store_true",
@@ -704,6 +818,8 @@ def main():
                     help="run only the linear-attention backward at 720p/5s")
     ap.add_argument("--sparse-only", action="store_true",
                     help="run only the block-sparse anchor at 720p/5s (25%% of the key tiles)")
+    ap.add_argument("--mx-only", action="store_true",
+                    help="run only the MX projection of the 720p QKVG shape")
     ap.add_argument("--chunk-only", action="store_true",
                     help="run only the 720p/60s block-causal chunk step (K steps back to back)")
     args = ap.parse_args()
@@ -726,6 +842,9 @@ def main():
             return
         if args.chunk_only:
             run_chunk_only(args)
+            return
+        if args.mx_only:
+            run_mx_only(args)
             return
         if args.impl == "reference":
             run_reference(args, world, rank)

@@ -206,12 +206,49 @@ SANA_API sana_status sana_linattn_block_causal_scan(const sana_shape* shape, int
  *   all N keys of the same batch entry and head.
  * rope may be NULL (no rotation).  scale <= 0 selects 1/sqrt(D).  Workspace:
  * sana_softmax_anchor_workspace_size() bytes (rotated Q and K copies).
+ * Accuracy domain (bf16): the rotated operands are rounded to bf16 before
+ * QK^T, so each logit carries an error of about 2^-9 of its own size and the
+ * output error grows with the spread of the scaled logits q.k * scale.  With
+ * Q, K ~ N(0, s^2) style inputs (logit standard deviation s) the max relative
+ * error against the float64 oracle measured 4.4e-3 (s = 1), 8.1e-3 (s = 4),
+ * 1.9e-2 (s = 8) and 3.1e-2 (s = 16): the 2e-2 parity bar holds for a logit
+ * standard deviation up to 8.  (The stack's anchors read RMS-normalised
+ * inputs through N(0, 1/C) projections: standard deviation about 1.)
  * ------------------------------------------------------------------------- */
 SANA_API size_t sana_softmax_anchor_workspace_size(const sana_shape* shape, sana_dtype dtype);
 SANA_API sana_status sana_softmax_anchor_fwd(const sana_shape* shape, sana_dtype dtype, const void* q,
                                     const void* k, const void* v, const void* gate_logits,
                                     const sana_rope* rope, float scale, void* out, void* ws,
                                     size_t ws_bytes, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The anchor's two phases, exposed so that each can be timed and reused
+ * (sana_softmax_anchor_fwd runs exactly these: sana_rope_apply on Q with
+ * mul = scale * log2(e) and on K with mul = 1, then the attention kernel).
+ *
+ * sana_rope_apply: out = mul * RoPE(x) for a (B, N, heads, head_dim) tensor,
+ * the 3D RoPE of the anchor reading ("SANA-Video" paper notes sec. 3.2: 3D
+ * RoPE; the pair layout as for the linear attention); rope == NULL applies no
+ * rotation (out = mul * x).  bf16 (head_dim 128) or fp32; out must not
+ * overlap x.  Shapes as sana_linattn_fwd.
+ *
+ * sana_softmax_anchor_rotated_fwd: Y = sigmoid(G) * softmax_2(Q' K'^T) V per
+ * (batch, head), bidirectional over all N keys ("SANA-Video 2.0" abstract:
+ * gated softmax anchors), where softmax_2 normalises 2^(logit) and Q', K' are
+ * the rotated operands (Q' = scale * log2(e) * RoPE(Q), K' = RoPE(K), as
+ * sana_rope_apply writes them), so the result equals sana_softmax_anchor_fwd.
+ * bf16 only, head_dim 128; gate_logits nullable; out must not alias an input.
+ * No workspace.  The bf16 rounding of Q' and K' bounds the accuracy: the 2e-2
+ * parity bar holds for scaled logits (q.k/sqrt(D)) with a standard deviation
+ * up to 8 (see sana_softmax_anchor_fwd).
+ * ------------------------------------------------------------------------- */
+SANA_API sana_status sana_rope_apply(const sana_shape* shape, sana_dtype dtype, const void* x,
+                                     const sana_rope* rope, float mul, void* out,
+                                     sana_stream_t stream);
+SANA_API sana_status sana_softmax_anchor_rotated_fwd(const sana_shape* shape, const void* q_rot,
+                                                     const void* k_rot, const void* v,
+                                                     const void* gate_logits, void* out,
+                                                     sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Block-sparse gated softmax anchor ([SV2] Experiments and [SV2a]: the
@@ -291,6 +328,49 @@ SANA_API sana_status sana_rmsnorm(long long rows, int C, sana_dtype dtype, const
                          void* y, sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * MX block-scaled projection GEMM ("SANA-Video 2.0" hyper.ai summary,
+ * Experiments: low-precision inference quantises only the linear GEMM layers,
+ * weights to MXFP4 and activations to MXFP8; attention stays bf16).  The
+ * formats are the OCP Microscaling v1.0 ones (a reading: the pages name them
+ * without defining them): blocks of 32 elements along K share one E8M0 scale
+ * 2^s, s = floor(log2 max|x|) - emax (8 for E4M3, 2 for E2M1) clamped to
+ * [-127, 127] (-127 for an all-zero block); elements x / 2^s rounded to
+ * nearest even and saturated.
+ *
+ * Layouts (device memory, caller-owned):
+ *   E4M3 codes: one byte per element, [rows][K] row-major;
+ *   E2M1 codes: two per byte, element 2i in the low nibble, [rows][K/2];
+ *   scales: sana_mx_scale_bytes(rows, K) bytes of E8M0 (s + 127) in 512-byte
+ *     atoms, one per 128 rows x 128 K-elements, ordered [ceil(rows/128)][K/128];
+ *     inside an atom, row r and 32-element block b (0..3) sit at byte
+ *     16 (r % 32) + 4 (r / 32) + b.  Padding rows hold scale 0.
+ *
+ * sana_mx_quantize: x bf16 (rows, K) -> codes q (E4M3 if fp4 == 0, E2M1 if
+ *   fp4 == 1) and scales.  K must be a positive multiple of 128.
+ * sana_mx_gemm: out[M][N] (bf16, row stride ldo) = epilogue(Q8(x) . Q4(w)^T)
+ *   from E4M3 activations (M, K) and E2M1 weights (N, K) with their scales,
+ *   fp32 accumulation on tcgen05 (kind::mxf8f6f4 with block scales);
+ *   epilogue as sana_gemm_bf16 (0 identity, 1 SiLU, 2 out += result).  N and
+ *   K positive multiples of 128; the E2M1 weights 32-byte aligned, the other
+ *   pointers 16-byte aligned.
+ * sana_mx_linear: the quantised projection of bf16 activations: quantises x
+ *   into the workspace (sana_mx_linear_workspace_size bytes, 256-byte
+ *   aligned) and runs sana_mx_gemm against pre-quantised weights.
+ * Errors: SANA_ERR_UNSUPPORTED for sizes the kernels do not cover,
+ * SANA_ERR_INVALID_ARG for NULL, misaligned or aliasing buffers.
+ * ------------------------------------------------------------------------- */
+SANA_API size_t sana_mx_scale_bytes(long long rows, int K);
+SANA_API sana_status sana_mx_quantize(const void* x, long long rows, int K, int fp4, void* q,
+                                      void* scales, sana_stream_t stream);
+SANA_API sana_status sana_mx_gemm(long long M, int N, int K, const void* xq,
+                                  const void* x_scales, const void* wq, const void* w_scales,
+                                  void* out, long long ldo, int epilogue, sana_stream_t stream);
+SANA_API size_t sana_mx_linear_workspace_size(long long M, int K);
+SANA_API sana_status sana_mx_linear(long long M, int N, int K, const void* x, const void* wq,
+                                    const void* w_scales, void* out, long long ldo, int epilogue,
+                                    void* ws, size_t ws_bytes, sana_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Hybrid stack forward ([SV2] method; [SV2a] 3:1 interleave).
  * Layer l (0-based) is a softmax anchor iff l % ratio == ratio - 1, else a
  * gated linear-attention layer.  Each layer has an attention sublayer
@@ -327,6 +407,35 @@ typedef struct {
 } sana_stack_weights;
 
 SANA_API size_t sana_hybrid_stack_workspace_size(const sana_shape* shape, const sana_stack_config* cfg);
+
+/* Where sana_hybrid_stack_fwd keeps its intermediates inside the workspace,
+ * as byte offsets from the workspace base (every tensor bf16, row-major,
+ * B*N rows).  Once a call has completed on its stream the workspace holds the
+ * state after its last layer L = cfg->layers - 1:
+ *   q, k, v, g  layer L's projections x_hat . W_qkvg^T, (B, N, C) each;
+ *   attn        layer L's gated attention output, before W_o, (B, N, C);
+ *   x_hat       the normalised input of layer L's last sublayer (its FFN
+ *               sublayer when ffn_mult > 0), (B, N, C);
+ *   ffn         SiLU(x_hat . W_up^T) of layer L, (B, N, ffn_mult*C);
+ *               SIZE_MAX when ffn_mult == 0;
+ *   blocks[i]   with AttnRes, block summary i for i < floor(layers /
+ *               block_span); the next buffer holds the running partial sum
+ *               when layers is not a multiple of block_span.  num_blocks
+ *               buffers in all (0 without AttnRes; then `out` holds the
+ *               residual stream).
+ * Running the stack for a prefix of its layers therefore exposes every
+ * sublayer's result; the layout depends only on shape and cfg->layers,
+ * block_span, ffn_mult and anchor_keep_tiles.  Returns SANA_ERR_INVALID_ARG
+ * for a NULL argument or a configuration sana_hybrid_stack_fwd rejects.
+ * (A testing and inspection aid: the pages define no such call.) */
+typedef struct {
+  size_t x_hat, q, k, v, g, attn, ffn;
+  int num_blocks;
+  size_t blocks[16];
+} sana_stack_ws_layout;
+SANA_API sana_status sana_hybrid_stack_workspace_layout(const sana_shape* shape,
+                                                        const sana_stack_config* cfg,
+                                                        sana_stack_ws_layout* layout);
 SANA_API sana_status sana_hybrid_stack_fwd(const sana_shape* shape, const sana_stack_config* cfg,
                                   const sana_stack_weights* weights, const sana_rope* rope,
                                   const void* x_embed, void* out, void* ws, size_t ws_bytes,

@@ -687,3 +687,16 @@ def max_rel_err(got, ref):
     if denom == 0.0:
         return float(np.max(np.abs(got)))
     return float(np.max(np.abs(got - ref)) / denom)
+
+
+def elementwise_rel_err(got, ref, floor=1e-3):
+    """max_i |got_i - ref_i| / max(|ref_i|, floor * max_j |ref_j|): the
+    elementwise companion of max_rel_err, which also sees errors in outputs
+    far smaller than the tensor's largest (e.g. elements gated towards 0)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    a = np.abs(ref)
+    m = np.max(a) if a.size else 0.0
+    if m == 0.0:
+        return float(np.max(np.abs(got))) if got.size else 0.0
+    return float(np.max(np.abs(got - ref) / np.maximum(a, floor * m)))

@@ -6,10 +6,12 @@ csrc/); this package is a thin ctypes binding over it.
 
 from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_route,
                    attnres_route_bwd, check,
-                   gemm_bf16, host_rope_tables, hybrid_stack_fwd, last_error, lib,
+                   gemm_bf16, host_rope_tables, hybrid_stack_fwd, hybrid_stack_workspace_size,
+                   hybrid_stack_workspace_views, last_error, lib,
                    linattn_apply, linattn_bwd, linattn_block_causal_scan, linattn_block_causal_scan_workspace_size,
                    linattn_block_causal_step, linattn_fwd, linattn_state,
-                   linattn_workspace_size, rmsnorm,
+                   linattn_workspace_size, mx_gemm, mx_linear, mx_quantize, rmsnorm, rope_apply,
+                   softmax_anchor_rotated_fwd,
                    anchor_tile_count, softmax_anchor_fwd, softmax_anchor_sparse_fwd,
                    softmax_anchor_sparse_workspace_size, stack_config,
                    sync_status)
@@ -17,9 +19,11 @@ from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_ro
 __all__ = [
     "EPI_NONE", "EPI_RESIDUAL", "EPI_SILU", "Rope", "SanaError", "attnres_route",
     "attnres_route_bwd", "check",
-    "gemm_bf16", "host_rope_tables", "hybrid_stack_fwd", "last_error", "lib",
+    "gemm_bf16", "host_rope_tables", "hybrid_stack_fwd", "hybrid_stack_workspace_size",
+    "hybrid_stack_workspace_views", "last_error", "lib",
     "linattn_apply", "linattn_bwd", "linattn_block_causal_scan", "linattn_block_causal_scan_workspace_size",
     "linattn_block_causal_step", "linattn_fwd", "linattn_state", "linattn_workspace_size", "rmsnorm",
+    "mx_gemm", "mx_linear", "mx_quantize", "rope_apply", "softmax_anchor_rotated_fwd",
     "anchor_tile_count", "softmax_anchor_fwd", "softmax_anchor_sparse_fwd",
     "softmax_anchor_sparse_workspace_size", "stack_config",
     "sync_status",

@@ -55,6 +55,12 @@ class StackWeights(Structure):
                 ("w_attn", c_void_p), ("w_ffn", c_void_p)]
 
 
+class StackWsLayout(Structure):
+    _fields_ = [("x_hat", c_size_t), ("q", c_size_t), ("k", c_size_t), ("v", c_size_t),
+                ("g", c_size_t), ("attn", c_size_t), ("ffn", c_size_t), ("num_blocks", c_int),
+                ("blocks", c_size_t * 16)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libsana.so not built ({LIB_PATH}); run softmax_attention_sana_b200/build.py")
@@ -93,6 +99,10 @@ def _load():
         "sana_softmax_anchor_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, POINTER(RopeStruct), c_float, c_void_p,
                                             c_void_p, c_size_t, c_void_p]),
+        "sana_rope_apply": (c_int, [POINTER(Shape), c_int, c_void_p, POINTER(RopeStruct), c_float,
+                                    c_void_p, c_void_p]),
+        "sana_softmax_anchor_rotated_fwd": (c_int, [POINTER(Shape), c_void_p, c_void_p, c_void_p,
+                                                    c_void_p, c_void_p, c_void_p]),
         "sana_softmax_anchor_sparse_workspace_size": (c_size_t, [POINTER(Shape), c_int]),
         "sana_softmax_anchor_sparse_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p,
                                                    c_void_p, c_void_p, POINTER(RopeStruct),
@@ -108,9 +118,19 @@ def _load():
                                    c_void_p, c_longlong, c_int, c_void_p]),
         "sana_rmsnorm": (c_int, [c_longlong, c_int, c_int, c_void_p, c_float, c_void_p, c_void_p]),
         "sana_hybrid_stack_workspace_size": (c_size_t, [POINTER(Shape), POINTER(StackConfig)]),
+        "sana_hybrid_stack_workspace_layout": (c_int, [POINTER(Shape), POINTER(StackConfig),
+                                                       POINTER(StackWsLayout)]),
         "sana_hybrid_stack_fwd": (c_int, [POINTER(Shape), POINTER(StackConfig),
                                           POINTER(StackWeights), POINTER(RopeStruct), c_void_p,
                                           c_void_p, c_void_p, c_size_t, c_void_p]),
+        "sana_mx_scale_bytes": (c_size_t, [c_longlong, c_int]),
+        "sana_mx_quantize": (c_int, [c_void_p, c_longlong, c_int, c_int, c_void_p, c_void_p,
+                                     c_void_p]),
+        "sana_mx_gemm": (c_int, [c_longlong, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                 c_void_p, c_longlong, c_int, c_void_p]),
+        "sana_mx_linear_workspace_size": (c_size_t, [c_longlong, c_int]),
+        "sana_mx_linear": (c_int, [c_longlong, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                   c_void_p, c_longlong, c_int, c_void_p, c_size_t, c_void_p]),
         "sana_sync_status": (c_int, [c_void_p]),
         "sana_selftest_bounded_wait": (c_int, [ctypes.c_uint, c_void_p]),
     }
@@ -343,6 +363,33 @@ def softmax_anchor_fwd(q, k, v, gate, rope, grid, heads, scale=0.0, out=None, ws
     return out
 
 
+def rope_apply(x, rope, grid, heads, mul=1.0, out=None):
+    """out = mul * RoPE(x) for a (B, N, C) tensor (rope may be None: no rotation)."""
+    _need(x, "x")
+    B, N, C = x.shape
+    s = make_shape(B, grid, heads, C // heads)
+    if out is None:
+        out = torch.empty_like(x)
+    check(lib.sana_rope_apply(ctypes.byref(s), _dtype_code(x), _ptr(x),
+                              None if rope is None else ctypes.byref(rope.struct), mul, _ptr(out),
+                              _stream()))
+    return out
+
+
+def softmax_anchor_rotated_fwd(q_rot, k_rot, v, gate, grid, heads, out=None):
+    """The anchor's attention phase on rotated operands (bf16): Q' = scale *
+    log2(e) * RoPE(Q), K' = RoPE(K) as rope_apply writes them."""
+    for t, n in ((q_rot, "q_rot"), (k_rot, "k_rot"), (v, "v")):
+        _need(t, n)
+    B, N, C = q_rot.shape
+    s = make_shape(B, grid, heads, C // heads)
+    if out is None:
+        out = torch.empty_like(v)
+    check(lib.sana_softmax_anchor_rotated_fwd(ctypes.byref(s), _ptr(q_rot), _ptr(k_rot), _ptr(v),
+                                              _ptr(gate), _ptr(out), _stream()))
+    return out
+
+
 def anchor_tile_count(N: int) -> int:
     """Key tiles of 128 tokens; query blocks are pairs of them."""
     return (N + 127) // 128
@@ -472,6 +519,73 @@ def hybrid_stack_fwd(x, weights, w_attn, w_ffn, rope: Rope, grid, heads, cfg: St
     check(lib.sana_hybrid_stack_fwd(ctypes.byref(s), ctypes.byref(cfg), ctypes.byref(sw),
                                     ctypes.byref(rope.struct), _ptr(x), _ptr(out), _ptr(ws),
                                     ws.numel(), _stream()))
+    return out
+
+
+def hybrid_stack_workspace_size(B, grid, heads, cfg: StackConfig, head_dim=128) -> int:
+    s = make_shape(B, grid, heads, head_dim)
+    return lib.sana_hybrid_stack_workspace_size(ctypes.byref(s), ctypes.byref(cfg))
+
+
+def hybrid_stack_workspace_views(ws, B, grid, heads, cfg: StackConfig, head_dim=128) -> dict:
+    """Views of the stack's intermediates inside its workspace `ws` (a uint8
+    tensor) after a call: keys x_hat, q, k, v, g, attn, ffn (absent when
+    ffn_mult is 0) and blocks (list), each (B, N, width) bf16."""
+    s = make_shape(B, grid, heads, head_dim)
+    lay = StackWsLayout()
+    check(lib.sana_hybrid_stack_workspace_layout(ctypes.byref(s), ctypes.byref(cfg),
+                                                 ctypes.byref(lay)))
+    N = grid[0] * grid[1] * grid[2]
+    C = heads * head_dim
+
+    def view(off, width):
+        nbytes = B * N * width * 2
+        return ws[off:off + nbytes].view(torch.bfloat16).view(B, N, width)
+
+    out = {k: view(getattr(lay, k), C) for k in ("x_hat", "q", "k", "v", "g", "attn")}
+    if cfg.ffn_mult > 0:
+        out["ffn"] = view(lay.ffn, cfg.ffn_mult * C)
+    out["blocks"] = [view(lay.blocks[i], C) for i in range(lay.num_blocks)]
+    return out
+
+
+# ---------------------------------------------------------------- MX projection GEMM
+
+def mx_quantize(x, fp4=False):
+    """MX quantisation of a bf16 (rows, K) tensor along K: returns (codes,
+    scales) as uint8 tensors -- E4M3 codes (rows, K), or E2M1 codes packed two
+    per byte (rows, K/2) with fp4, and the E8M0 scale atoms."""
+    _need(x, "x")
+    K = x.shape[-1]
+    rows = x.numel() // K
+    q = torch.empty(rows, K // 2 if fp4 else K, dtype=torch.uint8, device=x.device)
+    sf = torch.empty(max(int(lib.sana_mx_scale_bytes(rows, K)), 16), dtype=torch.uint8,
+                     device=x.device)
+    check(lib.sana_mx_quantize(_ptr(x), rows, K, int(bool(fp4)), _ptr(q), _ptr(sf), _stream()))
+    return q, sf
+
+
+def mx_gemm(xq, x_scales, wq, w_scales, N, out=None, epilogue=EPI_NONE):
+    """out = epilogue(Q8(x) . Q4(w)^T) from quantised operands (see mx_quantize)."""
+    M, K = xq.shape
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=xq.device)
+    check(lib.sana_mx_gemm(M, N, K, _ptr(xq), _ptr(x_scales), _ptr(wq), _ptr(w_scales), _ptr(out),
+                           out.stride(0), epilogue, _stream()))
+    return out
+
+
+def mx_linear(x, wq, w_scales, N, out=None, epilogue=EPI_NONE, ws=None):
+    """The quantised projection of bf16 activations x (M, K) against
+    pre-quantised MXFP4 weights: activations quantised to MXFP8 on the fly."""
+    _need(x, "x")
+    M, K = x.shape
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = _ws(lib.sana_mx_linear_workspace_size(M, K), x.device)
+    check(lib.sana_mx_linear(M, N, K, _ptr(x), _ptr(wq), _ptr(w_scales), _ptr(out), out.stride(0),
+                             epilogue, _ptr(ws), ws.numel(), _stream()))
     return out
 
 

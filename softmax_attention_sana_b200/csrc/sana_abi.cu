@@ -119,6 +119,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 }  // namespace
 
+bool make_tmap_2d_typed(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                        uint64_t cols, uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols,
+                        uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                        uint64_t batches, uint64_t row_stride, uint64_t batch_stride,
                        uint32_t box_rows) {
@@ -718,6 +732,42 @@ sana_status sana_softmax_anchor_fwd(const sana_shape* s, sana_dtype dt, const vo
   return anchor_run(*s, dt, q, k, v, g, rope ? &rd : nullptr, scale, out, ws, ws_bytes, stream);
 }
 
+sana_status sana_rope_apply(const sana_shape* s, sana_dtype dt, const void* x,
+                           const sana_rope* rope, float mul, void* out, sana_stream_t stream) {
+  const char* who = "sana_rope_apply";
+  if (sana_status e = check_shape(s, dt, who)) return e;
+  if (rope)
+    if (sana_status e = check_rope(rope, s, who)) return e;
+  if (!std::isfinite(mul)) return fail(SANA_ERR_INVALID_ARG, "%s: mul is not finite", who);
+  if (s->T == 0) return SANA_OK;
+  if (!x || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  if (!aligned16(x) || !aligned16(out))
+    return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * esize(dt);
+  if (overlap(out, n, x, n)) return fail(SANA_ERR_INVALID_ARG, "%s: out aliases x", who);
+  RopeDev rd{};
+  if (rope) rd = to_dev(*rope);
+  return rope_rotate_run(x, dt == SANA_BF16, rope ? &rd : nullptr, to_grid(*s), s->B,
+                         s->head_dim, mul, out, stream);
+}
+
+sana_status sana_softmax_anchor_rotated_fwd(const sana_shape* s, const void* q_rot,
+                                            const void* k_rot, const void* v, const void* g,
+                                            void* out, sana_stream_t stream) {
+  const char* who = "sana_softmax_anchor_rotated_fwd";
+  if (sana_status e = check_shape(s, SANA_BF16, who)) return e;
+  if (s->T == 0) return SANA_OK;
+  if (!q_rot || !k_rot || !v || !out) return fail(SANA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  const void* ptrs[5] = {q_rot, k_rot, v, g, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t n = (size_t)s->B * s->T * s->H * s->W * s->heads * s->head_dim * 2;
+  if (overlap(out, n, q_rot, n) || overlap(out, n, k_rot, n) || overlap(out, n, v, n) ||
+      overlap(out, n, g, n))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an input", who);
+  return anchor_bf16_run(*s, q_rot, k_rot, v, g, to_grid(*s), nullptr, 0, out, stream);
+}
+
 size_t sana_softmax_anchor_sparse_workspace_size(const sana_shape* s, sana_dtype dt) {
   if (check_shape(s, dt, "sana_softmax_anchor_sparse_workspace_size") != SANA_OK ||
       dt != SANA_BF16)
@@ -849,6 +899,79 @@ sana_status sana_gemm_bf16(long long M, int N, int K, const void* A, long long l
   if (epilogue < 0 || epilogue > 2) return fail(SANA_ERR_INVALID_ARG, "%s: bad epilogue %d", who, epilogue);
   if (!aligned16(A) || !aligned16(W) || !aligned16(out)) return fail(SANA_ERR_INVALID_ARG, "%s: pointers not 16-byte aligned", who);
   return gemm_run(M, N, K, A, lda, W, out, ldo, epilogue, stream);
+}
+
+// ---------------------------------------------------------------- MX projection GEMM
+size_t sana_mx_scale_bytes(long long rows, int K) {
+  if (rows < 0 || K < 128 || K % 128 != 0) return 0;
+  return mx_scale_bytes(rows, K);
+}
+
+sana_status sana_mx_quantize(const void* x, long long rows, int K, int fp4, void* q, void* scales,
+                             sana_stream_t stream) {
+  const char* who = "sana_mx_quantize";
+  if (rows < 0 || K < 128 || K % 128 != 0 || (fp4 != 0 && fp4 != 1))
+    return fail(SANA_ERR_INVALID_ARG, "%s: needs rows >= 0, K a positive multiple of 128, fp4 0/1",
+                who);
+  if (rows == 0) return SANA_OK;
+  if (!x || !q || !scales) return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned16(x) || !aligned16(q) || !aligned16(scales))
+    return fail(SANA_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  const size_t nx = (size_t)rows * K * 2, nq = (size_t)rows * K / (fp4 ? 2 : 1);
+  const size_t ns = mx_scale_bytes(rows, K);
+  if (overlap(q, nq, x, nx) || overlap(scales, ns, x, nx) || overlap(scales, ns, q, nq))
+    return fail(SANA_ERR_INVALID_ARG, "%s: buffers overlap", who);
+  return mx_quantize_run(x, rows, K, fp4 != 0, q, scales, stream);
+}
+
+sana_status sana_mx_gemm(long long M, int N, int K, const void* xq, const void* x_scales,
+                         const void* wq, const void* w_scales, void* out, long long ldo,
+                         int epilogue, sana_stream_t stream) {
+  const char* who = "sana_mx_gemm";
+  if (M < 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: needs N and K positive multiples of 128 (N=%d K=%d)",
+                who, N, K);
+  if (ldo < N || ldo % 8 != 0) return fail(SANA_ERR_INVALID_ARG, "%s: ldo must be >= N and a multiple of 8", who);
+  if (epilogue < 0 || epilogue > 2) return fail(SANA_ERR_INVALID_ARG, "%s: bad epilogue %d", who, epilogue);
+  if (M == 0) return SANA_OK;
+  if (!xq || !x_scales || !wq || !w_scales || !out)
+    return fail(SANA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned16(xq) || !aligned16(x_scales) || !aligned16(w_scales) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(wq) & 31u))
+    return fail(SANA_ERR_INVALID_ARG,
+                "%s: pointers must be 16-byte aligned (the E2M1 weights 32-byte aligned)", who);
+  const size_t no = (size_t)M * ldo * 2;
+  if (overlap(out, no, xq, (size_t)M * K) || overlap(out, no, wq, (size_t)N * K / 2) ||
+      overlap(out, no, x_scales, mx_scale_bytes(M, K)) ||
+      overlap(out, no, w_scales, mx_scale_bytes(N, K)))
+    return fail(SANA_ERR_INVALID_ARG, "%s: out aliases an operand", who);
+  return mx_gemm_run(M, N, K, xq, x_scales, wq, w_scales, out, ldo, epilogue, stream);
+}
+
+size_t sana_mx_linear_workspace_size(long long M, int K) {
+  if (M < 0 || K < 128 || K % 128 != 0) return 0;
+  return align_up((size_t)M * K, 256) + align_up(mx_scale_bytes(M, K), 256);
+}
+
+sana_status sana_mx_linear(long long M, int N, int K, const void* x, const void* wq,
+                           const void* w_scales, void* out, long long ldo, int epilogue, void* ws,
+                           size_t ws_bytes, sana_stream_t stream) {
+  const char* who = "sana_mx_linear";
+  if (M < 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
+    return fail(SANA_ERR_UNSUPPORTED, "%s: needs N and K positive multiples of 128 (N=%d K=%d)",
+                who, N, K);
+  if (M == 0) return SANA_OK;
+  const size_t need = sana_mx_linear_workspace_size(M, K);
+  if (!ws || ws_bytes < need)
+    return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  if (out && overlap(ws, need, out, (size_t)M * ldo * 2))
+    return fail(SANA_ERR_INVALID_ARG, "%s: workspace aliases the output", who);
+  char* xq = static_cast<char*>(ws);
+  char* xs = xq + align_up((size_t)M * K, 256);
+  if (sana_status e = sana_mx_quantize(x, M, K, 0, xq, xs, stream)) return e;
+  return sana_mx_gemm(M, N, K, xq, xs, wq, w_scales, out, ldo, epilogue, stream);
 }
 
 sana_status sana_selftest_bounded_wait(unsigned int limit_ms, sana_stream_t stream) {

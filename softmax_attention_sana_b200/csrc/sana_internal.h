@@ -53,6 +53,12 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols, uint64
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                        uint64_t row_stride, uint32_t box_cols, uint32_t box_rows);
 
+// 2D view of a (rows, cols) tensor of any TMA element type, 128-byte swizzle;
+// row stride in bytes; box = (box_cols elements, box_rows rows).
+bool make_tmap_2d_typed(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                        uint64_t cols, uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols,
+                        uint32_t box_rows);
+
 // Grid of one call, as the kernels see it.  Batch entry b covers frames
 // [t_offset + b * t_stride, + T): t_stride is 0 for independent sequences and
 // the block length when consecutive blocks of one sequence are batched.
@@ -186,5 +192,16 @@ sana_status rmsnorm_run(long long rows, int C, sana_dtype dt, const void* x, flo
                         cudaStream_t st);
 sana_status gemm_run(long long M, int N, int K, const void* A, long long lda, const void* W,
                      void* out, long long ldo, int epilogue, cudaStream_t st);
+
+// ---------------------------------------------------------------- MX projection GEMM
+// Scale bytes of a (rows, K) operand: 512-byte atoms of 128 rows x 128 K-elements.
+size_t mx_scale_bytes(long long rows, int K);
+// bf16 (rows, K) -> E4M3 bytes (fp4 = false) or packed E2M1 (fp4 = true) + scales.
+sana_status mx_quantize_run(const void* x, long long rows, int K, bool fp4, void* q, void* sf,
+                            cudaStream_t st);
+// out[M][N] = epilogue(Q8(x) . Q4(w)^T) from quantised operands.
+sana_status mx_gemm_run(long long M, int N, int K, const void* xq, const void* xsf,
+                        const void* wq, const void* wsf, void* out, long long ldo, int epilogue,
+                        cudaStream_t st);
 
 }  // namespace sana

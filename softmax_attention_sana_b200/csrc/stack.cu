@@ -19,6 +19,7 @@
 //   u . W_down^T             -> partial +=       (GEMM, residual epilogue)
 //   every block_span layers: partial becomes a summary (pointer hand-over).
 #include <cmath>
+#include <cstdint>
 #include <vector>
 
 #include "sana_common.cuh"
@@ -98,6 +99,29 @@ using namespace sana;
 extern "C" size_t sana_hybrid_stack_workspace_size(const sana_shape* s, const sana_stack_config* c) {
   if (check_cfg(s, c) != SANA_OK) return 0;
   return carve_stack(*s, *c, nullptr).bytes;
+}
+
+extern "C" sana_status sana_hybrid_stack_workspace_layout(const sana_shape* s,
+                                                          const sana_stack_config* c,
+                                                          sana_stack_ws_layout* out) {
+  if (!out) return fail(SANA_ERR_INVALID_ARG, "stack layout: NULL output");
+  if (sana_status e = check_cfg(s, c)) return e;
+  // carve from a fake non-null base so that the offsets come out directly
+  char* const base = reinterpret_cast<char*>(256);
+  const StackWs w = carve_stack(*s, *c, base);
+  auto off = [&](const void* p) { return static_cast<size_t>(static_cast<const char*>(p) - base); };
+  sana_stack_ws_layout L{};
+  L.x_hat = off(w.xhat);
+  L.q = off(w.q);
+  L.k = off(w.k);
+  L.v = off(w.v);
+  L.g = off(w.g);
+  L.attn = off(w.attn);
+  L.ffn = w.ffn ? off(w.ffn) : SIZE_MAX;
+  L.num_blocks = static_cast<int>(w.blocks.size());
+  for (int i = 0; i < L.num_blocks; ++i) L.blocks[i] = off(w.blocks[i]);
+  *out = L;
+  return SANA_OK;
 }
 
 extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_stack_config* c,

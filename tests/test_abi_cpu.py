@@ -186,3 +186,67 @@ def test_attnres_and_gemm_validation():
         == L.SANA_ERR_UNSUPPORTED
     assert L.lib.sana_gemm_bf16(128, 128, 100, 4096, 100, 8192, 1 << 20, 128, 0, None) \
         == L.SANA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("layers,span,attnres,ffn", [(16, 8, True, 3), (4, 8, False, 0),
+                                                      (5, 2, True, 0), (8, 8, True, 3)])
+def test_stack_workspace_layout_is_disjoint_and_inside_the_workspace(layers, span, attnres, ffn):
+    """The intermediates the stack exposes lie inside its workspace, do not
+    overlap, and there is one AttnRes buffer per started block."""
+    grid, heads = (21, 45, 80), 24
+    cfg = sana.stack_config(layers, block_span=span, use_attnres=attnres, ffn_mult=ffn)
+    s = _lib.make_shape(1, grid, heads, 128)
+    lay = _lib.StackWsLayout()
+    assert _lib.lib.sana_hybrid_stack_workspace_layout(ctypes.byref(s), ctypes.byref(cfg),
+                                                       ctypes.byref(lay)) == _lib.SANA_OK
+    total = _lib.lib.sana_hybrid_stack_workspace_size(ctypes.byref(s), ctypes.byref(cfg))
+    tok_bytes = grid[0] * grid[1] * grid[2] * heads * 128 * 2
+    spans = [(getattr(lay, k), tok_bytes) for k in ("x_hat", "q", "k", "v", "g", "attn")]
+    if ffn:
+        spans.append((lay.ffn, ffn * tok_bytes))
+    else:
+        assert lay.ffn == 2 ** 64 - 1
+    nblocks = -(-layers // span) if attnres else 0
+    assert lay.num_blocks == nblocks
+    spans += [(lay.blocks[i], tok_bytes) for i in range(nblocks)]
+    spans.sort()
+    for (a, na), (b, _) in zip(spans, spans[1:]):
+        assert a + na <= b
+    assert spans[-1][0] + spans[-1][1] <= total
+    assert all(off % 256 == 0 for off, _ in spans)
+
+
+def test_stack_workspace_layout_rejects_bad_arguments():
+    cfg = sana.stack_config(4, block_span=8, use_attnres=False, ffn_mult=0)
+    s = _lib.make_shape(1, (2, 4, 8), 2, 128)
+    assert _lib.lib.sana_hybrid_stack_workspace_layout(ctypes.byref(s), ctypes.byref(cfg),
+                                                       None) == _lib.SANA_ERR_INVALID_ARG
+    bad = sana.stack_config(0, block_span=8)
+    lay = _lib.StackWsLayout()
+    assert _lib.lib.sana_hybrid_stack_workspace_layout(ctypes.byref(s), ctypes.byref(bad),
+                                                       ctypes.byref(lay)) != _lib.SANA_OK
+
+
+def test_mx_sizes_and_validation():
+    """The MX projection's scale-atom sizes and argument checks (no device
+    work: every call below fails validation first)."""
+    L = _lib
+    # 75,600 rows x 3072: 591 row atoms x 24 K atoms x 512 bytes
+    assert L.lib.sana_mx_scale_bytes(75600, 3072) == 591 * 24 * 512
+    assert L.lib.sana_mx_scale_bytes(1, 128) == 512
+    assert L.lib.sana_mx_scale_bytes(10, 100) == 0
+    assert L.lib.sana_mx_linear_workspace_size(300, 256) >= 300 * 256 + 3 * 2 * 512
+    M = 1 << 20
+    assert L.lib.sana_mx_quantize(M, 10, 100, 0, 2 * M, 3 * M, None) == L.SANA_ERR_INVALID_ARG
+    assert L.lib.sana_mx_quantize(M, 10, 128, 2, 2 * M, 3 * M, None) == L.SANA_ERR_INVALID_ARG
+    assert L.lib.sana_mx_quantize(M + 8, 10, 128, 1, 2 * M, 3 * M, None) == L.SANA_ERR_INVALID_ARG
+    assert L.lib.sana_mx_quantize(M, 10, 128, 0, M, 3 * M, None) == L.SANA_ERR_INVALID_ARG
+    g = L.lib.sana_mx_gemm
+    assert g(256, 100, 256, M, 2 * M, 3 * M, 4 * M, 5 * M, 100, 0, None) == L.SANA_ERR_UNSUPPORTED
+    assert g(256, 128, 192, M, 2 * M, 3 * M, 4 * M, 5 * M, 128, 0, None) == L.SANA_ERR_UNSUPPORTED
+    assert g(256, 128, 256, M, 2 * M, 3 * M + 16, 4 * M, 5 * M, 128, 0, None) == \
+        L.SANA_ERR_INVALID_ARG and "32-byte" in L.last_error()
+    assert g(256, 128, 256, M, 2 * M, 3 * M, 4 * M, M, 128, 0, None) == L.SANA_ERR_INVALID_ARG
+    assert g(256, 128, 256, M, 2 * M, 3 * M, 4 * M, 5 * M, 128, 3, None) == L.SANA_ERR_INVALID_ARG
+    lin = L.lib.sana_mx_linear
+    assert lin(300, 256, 256, M, 2 * M, 3 * M, 4 * M, 256, 0, 5 * M, 64, None) == L.SANA_ERR_WORKSPACE

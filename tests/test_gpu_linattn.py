@@ -110,6 +110,22 @@ def full_size_sampled_check(wl, rows_count=768):
     return err
 
 
+@pytest.mark.parametrize("c", [-12.0, -8.0, -4.0, 6.0])
+def test_gate_relative_accuracy_at_saturated_logits(c):
+    """Every gate logit equal to c: the output is sigmoid(c) times the ungated
+    layer, so the parity measure (relative to the output's own largest value)
+    sees the gate's relative error even where sigmoid(c) is about 6e-6."""
+    grid, heads = (3, 8, 16), 2
+    N, C = 384, 256
+    q, k, v = (si.normal(7600 + i, (1, N, C)) for i in range(3))
+    g = torch.full((1, N, C), c, dtype=torch.bfloat16)
+    y = gpu_lin(q, k, v, g, grid, (22, 21, 21), heads).cpu()
+    yo, _, _ = orc.linattn_bidirectional(f64(q), f64(k), f64(v), grid, (22, 21, 21), heads,
+                                         gate=f64(g))
+    err = orc.max_rel_err(f64(y), yo)
+    assert err <= BF16_TOL, err
+
+
 def test_480p_full_size_sampled():
     full_size_sampled_check(si.P480)
 

@@ -169,3 +169,21 @@ def test_stack_full_size_runs_deterministically(layers, attnres, ffn):
     y2 = _run_stack(x, ws, w_attn, w_ffn, grid, wl.heads, cfg)
     assert torch.isfinite(y1.float()).all()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.slow
+def test_stack_full_width_and_depth_short_sequence():
+    """The 16-layer AttnRes stack at full width (24 heads x 128, hidden 3072,
+    FFN 3C) on a 512-token grid, against the whole float64 oracle stack: the
+    error accumulated over 32 sublayers of bf16 partial sums and residual
+    routes, end to end."""
+    grid, heads, layers = (2, 16, 16), 24, 16
+    C, N = heads * 128, 512
+    x, ws, w_attn, w_ffn = _stack_inputs(C, N, layers, 3, 15000 + layers)
+    cfg = sana.stack_config(layers, block_span=8, use_attnres=True, ffn_mult=3)
+    y = _run_stack(x, ws, w_attn, w_ffn, grid, heads, cfg)
+    yo = _oracle_stack(x, ws, w_attn, w_ffn, grid, heads, layers, 8, True, True)
+    err = orc.max_rel_err(f64(y), yo)
+    print(f"16-layer stack, N=512, C=3072: max_rel {err:.3e} "
+          f"elementwise {orc.elementwise_rel_err(f64(y), yo):.3e}")
+    assert err <= BF16_TOL, err

@@ -764,3 +764,17 @@ def test_mx_linear_is_the_product_of_the_dequantised_operands():
     qb = orc.mx_dequantize(*orc.mx_quantize(b, orc.E2M1))
     assert np.allclose(orc.mx_linear(a, b), qa @ qb.T, rtol=0, atol=1e-12)
     assert rel(orc.mx_linear(a, b), a @ b.T) < 0.5
+
+
+def test_error_measures_hand_worked():
+    """max_rel_err divides the largest difference by the largest reference
+    magnitude; elementwise_rel_err divides each difference by its own
+    reference magnitude, floored at 1e-3 of the largest."""
+    ref = np.array([10.0, 1.0, -0.001, 0.0])
+    got = np.array([10.5, 1.0, -0.002, 0.0])
+    assert orc.max_rel_err(got, ref) == pytest.approx(0.05, rel=1e-15)
+    # element 2: |0.001| / max(0.001, 0.01) = 0.1; element 0: 0.5 / 10 = 0.05
+    assert orc.elementwise_rel_err(got, ref) == pytest.approx(0.1, rel=1e-12)
+    got2 = np.array([10.0, 1.0, -0.001, 0.003])   # 0.003 / 0.01
+    assert orc.elementwise_rel_err(got2, ref) == pytest.approx(0.3, rel=1e-12)
+    assert orc.max_rel_err(got2, ref) == pytest.approx(0.0003, rel=1e-12)
