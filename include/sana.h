@@ -106,6 +106,10 @@ SANA_API sana_status sana_rope_bind(const float* tables_device, int T_total, int
  * sana_linattn_workspace_size() bytes (256-byte aligned), caller-owned,
  * contents undefined on return.  The state reduction over N is split across
  * CTAs and combined in a fixed order, so results are bit-reproducible.
+ * Gate precision (bf16): sigmoid(G) = 1/2 + tanh(G/2)/2 with the hardware
+ * tanh approximation, absolute error about 2.5e-4 -- a relative error below
+ * 1.5% for logits >= -4; for logits below -4 the gated output is under 2% of
+ * the ungated one and carries an error below 1e-3 of the ungated scale.
  * ------------------------------------------------------------------------- */
 SANA_API size_t sana_linattn_workspace_size(const sana_shape* shape, sana_dtype dtype);
 SANA_API sana_status sana_linattn_fwd(const sana_shape* shape, sana_dtype dtype, const void* q,

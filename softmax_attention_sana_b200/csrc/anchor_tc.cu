@@ -12,22 +12,13 @@
 //                   j: O_0 += P_0 V_j, S_0 = Q'_0 K'_{j+1}^T, O_1 += P_1 V_j,
 //                   S_1 = Q'_1 K'_{j+1}^T, so one warpgroup's softmax runs while
 //                   the tensor core works for the other
-//   8 softmax warps, all on each query tile in turn (tile 0, then tile 1,
-//                   for every key tile): warp w owns rows 32 (w % 4) .. + 31
-//                   (its TMEM lane quarter) and key columns 64 (w / 4) .. + 63,
-//                   so each row is shared by two threads that exchange their
-//                   partial maxima through shared memory (a bounded mbarrier
-//                   wait, no named barrier).  Each thread holds its 64 logits
-//                   in registers: row max, base-2 exponentials, P as bf16
-//                   written over the first 32 of its own 64 S columns, lazy
-//                   rescaling of its half of O in TMEM (only when the row max
-//                   grows by more than 2^8, decided warp-uniformly), and in the
-//                   epilogue 1/l, gate and its 64-column half of the Y tile.
-//                   Splitting rows over two threads halves the softmax latency
-//                   on the chain S_i -> softmax_i -> P_i V -> S_i of the next key
-//                   tile, which bounds the kernel more than the tensor core.
+//   2 x 4 softmax warps (thread = query row of its tile): row max, base-2
+//                   exponentials, P as bf16 written back over its S columns,
+//                   lazy rescaling of O in TMEM (only when a row's max grows
+//                   by more than 2^8, decided warp-uniformly), final 1/l, gate
+//                   and TMA store.
 // TMEM (512 columns): S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512);
-// P_i occupies columns [0, 32) and [64, 96) of S_i (keys 0-63 and 64-127).
+// P_i occupies the first 64 columns of S_i.
 //
 // Block-sparse form: with a tile list, the CTA walks only the `keep` key tiles
 // listed for its 256-query block (in list order) instead of all of them; the
@@ -130,8 +121,6 @@ struct AnchorCtl {
   uint64_t v_full[kVS], v_empty[kVS];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t ysync[2];  // the 128 output rows of tile i are staged (bounded wait)
-  uint64_t pair[2][4];  // the two threads of each row (warps w, w + 4) met, per tile
-  float red[2][2][2][kRows];  // [use parity][tile][half][row]: partial max, then row sum
   uint32_t tmem;
   int abort_flag;
 };
@@ -175,10 +164,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.s_full[i], 1);
-      mbar_init(&ctl.p_full[i], 256);
+      mbar_init(&ctl.p_full[i], 128);
       mbar_init(&ctl.pv_done[i], 1);
-      mbar_init(&ctl.ysync[i], 256);
-      for (int q = 0; q < 4; ++q) mbar_init(&ctl.pair[i][q], 64);
+      mbar_init(&ctl.ysync[i], 128);
     }
     ctl.abort_flag = 0;
     mbar_fence_init();
@@ -271,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bv = desc_advance(dv0, (j % kVS) * kTileB);
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk)
-          umma_ts(tmem + 256 + i * 128, tmem + i * 128 + (kk >> 2) * 64 + (kk & 3) * 8,
-                  desc_advance(bv, kk * 2048), idesc_o, (j | kk) != 0);
+          umma_ts(tmem + 256 + i * 128, tmem + i * 128 + kk * 8, desc_advance(bv, kk * 2048),
+                  idesc_o, (j | kk) != 0);
         umma_commit(&ctl.pv_done[i]);
       };
       bool ok = mbar_wait(&ctl.q_full, 0, wc, 0x33) && nk_all > 0 &&
@@ -311,46 +299,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------ softmax warps
-    const int half = warp >> 2;                 // key columns [64 half, 64 half + 64) of each tile
-    const int q4 = warp & 3;                    // TMEM lane quarter
-    const int r = q4 * 32 + lane;               // row within a query tile
-    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    // ------------------------------------------------ softmax warps: thread = query row
+    const int qi = warp >> 2;                 // which query tile
+    const int r = (warp & 3) * 32 + lane;     // row within the tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tmem_s = tmem + qi * 128, tmem_o = tmem + 256 + qi * 128;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // the two threads of a row swap one value through shared memory; the
-    // mbarrier of the warp pair completes one phase per use (bounded wait)
-    auto swap = [&](int qi, int use, float v) -> float {
-      float* slot = ctl.red[use & 1][qi][half];
-      slot[r] = v;
-      mbar_arrive(&ctl.pair[qi][q4]);
-      ok = mbar_wait(&ctl.pair[qi][q4], use & 1, wc, 0x3e) && ok;
-      return ctl.red[use & 1][qi][half ^ 1][r];
-    };
     for (int j = 0; ok && j < nk_all; ++j) {
+      // warp-uniform outcome: tcgen05.ld / st are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctl.s_full[qi], j & 1, wc, 0x38))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       const bool last = key_tile(j) == nkv - 1 && kv_tail < kRows;
-      for (int qi = 0; qi < 2; ++qi) {
-        const uint32_t tmem_s = tmem + qi * 128 + half * 64, tmem_o = tmem + 256 + qi * 128 + half * 64;
-        // warp-uniform outcome: tcgen05.ld / st are warp-collective
-        if (!__all_sync(0xffffffffu, mbar_wait(&ctl.s_full[qi], j & 1, wc, 0x38) && ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      // pass 1: row max, 64 columns in registers at a time (four independent
+      // chains of 3-input max)
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
         uint32_t sa[32], sb[32];
-        tmem_ld32(tmem_s + lane_base, sa);
-        tmem_ld32(tmem_s + lane_base + 32, sb);
+        tmem_ld32(tmem_s + lane_base + hh * 64, sa);
+        tmem_ld32(tmem_s + lane_base + hh * 64 + 32, sb);
         tmem_ld_wait();
         if (last) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (half * 64 + i >= kv_tail) sa[i] = __float_as_uint(-INFINITY);
-            if (half * 64 + 32 + i >= kv_tail) sb[i] = __float_as_uint(-INFINITY);
+            if (hh * 64 + i >= kv_tail) sa[i] = __float_as_uint(-INFINITY);
+            if (hh * 64 + 32 + i >= kv_tail) sb[i] = __float_as_uint(-INFINITY);
           }
         }
-        // partial row max (four independent chains of 3-input max), then the
-        // other half's through the swap
-        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 32; i += 8)
 #pragma unroll
@@ -361,28 +340,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int a = 0; a < 4; ++a)
             mq[a] = max3(mq[a], __uint_as_float(sa[i + 2 * a + 1]), __uint_as_float(sb[i + 2 * a]));
-        float mx = max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
-        mx = fmaxf(mx, swap(qi, j, mx));
-        const float m_new = fmaxf(m[qi], mx);
-        // lazy rescaling: a row moves its reference max only when the max grew
-        // by more than 2^8; both threads of a row decide alike, and the
-        // decision to touch O is warp-uniform because TMEM access is
-        // warp-collective (rows that keep their max use a factor 1).  A moved
-        // max is rounded up to an integer so that the folded constant of the
-        // FMA-pipe exponential (1.5 * 2^23 - m) is exact.
-        const bool grow = m_new > m[qi] + kRescaleLog2;
-        const bool any_grow = __any_sync(0xffffffffu, grow);
-        const float m_use = grow ? ceilf(m_new) : m[qi];
-        const float corr = ex2(m[qi] - m_use);  // 0 on the first tile
-        const uint64_t neg_m = pk2(-m_use, -m_use);
-        const uint64_t cfold = pk2(12582912.f - m_use, 12582912.f - m_use);
-        const float s_lo = m_use - 126.f;
-        uint64_t rs2 = pk2(0.f, 0.f);
-        uint32_t pk[32];
+      }
+      const float mx = max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      const float m_new = fmaxf(m, mx);
+      // lazy rescaling: a row moves its reference max only when the max grew
+      // by more than 2^8; the decision to touch O is warp-uniform because TMEM
+      // access is warp-collective (rows that keep their max use a factor 1).
+      // A moved max is rounded up to an integer so that the folded constant of
+      // the FMA-pipe exponential (1.5 * 2^23 - m) is exact.
+      const bool grow = m_new > m + kRescaleLog2;
+      const bool any_grow = __any_sync(0xffffffffu, grow);
+      const float m_use = grow ? ceilf(m_new) : m;
+      const float corr = ex2(m - m_use);  // 0 on the first tile
+      // pass 2: P = 2^(s - m) over 32-column chunks, the next chunk's load in
+      // flight while this one is exponentiated (MUFU for most pairs, the
+      // FMA-pipe polynomial for kEmuPairs of every 8).  P of chunk c goes to
+      // columns [16c, 16c + 16), inside S chunks already read.
+      const uint64_t neg_m = pk2(-m_use, -m_use);
+      const uint64_t cfold = pk2(12582912.f - m_use, 12582912.f - m_use);
+      const float s_lo = m_use - 126.f;
+      uint64_t rs2 = pk2(0.f, 0.f);
+      uint32_t sc[2][32];
+      uint32_t pk[32];
+      tmem_ld32(tmem_s + lane_base, sc[0]);
+      tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const uint32_t* src = i < 32 ? sa : sb;
-          const float s0 = __uint_as_float(src[i & 31]), s1 = __uint_as_float(src[(i & 31) + 1]);
+      for (int c = 0; c < 4; ++c) {
+        if (c < 3) tmem_ld32(tmem_s + lane_base + (c + 1) * 32, sc[(c + 1) & 1]);
+        uint32_t* cur = sc[c & 1];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float s0 = __uint_as_float(cur[i]), s1 = __uint_as_float(cur[i + 1]);
+          if (last) {
+            if (c * 32 + i >= kv_tail) s0 = -INFINITY;
+            if (c * 32 + i + 1 >= kv_tail) s1 = -INFINITY;
+          }
           float p0, p1;
           if (((i >> 1) & 7) >= 8 - kEmuPairs) {
             exp2_fma2(s0, s1, s_lo, cfold, p0, p1);
@@ -393,91 +385,84 @@ __global__ void __launch_bounds__(kThreads, 1)
             p1 = ex2(x1);
           }
           rs2 = add2(rs2, pk2(p0, p1));
-          pk[i >> 1] = f2_to_bf2(p0, p1);
+          pk[(c & 1) * 16 + i / 2] = f2_to_bf2(p0, p1);
         }
-        // P over the first 32 of this thread's 64 S columns (all of them are
-        // in registers already)
-        tmem_st32(tmem_s + lane_base, pk);
-        float rs0, rs1;
-        up2(rs2, rs0, rs1);
-        l[qi] = l[qi] * corr + (rs0 + rs1);
-        m[qi] = m_use;
-        if (any_grow && j >= 1) {
-          // O_i holds the sum over tiles < j (their PV MMAs finished before
-          // S_i of this tile was issued); scale this thread's half of it
-          // before the next PV accumulates
-          if (!__all_sync(0xffffffffu, mbar_wait(&ctl.pv_done[qi], (j - 1) & 1, wc, 0x39) && ok)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem_o + lane_base + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-            tmem_st32(tmem_o + lane_base + c * 32, o);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&ctl.p_full[qi]);
+        if (c & 1) tmem_st32(tmem_s + lane_base + (c >> 1) * 32, pk);
+        if (c < 3) tmem_ld_wait();
       }
-    }
-    // ---------------- epilogue: Y = O / l * sigmoid(G), this thread's 64 columns
-    if (kGate) ok = __all_sync(0xffffffffu, ok && mbar_wait(&ctl.g_full, 0, wc, 0x3d));
-    for (int qi = 0; qi < 2; ++qi) {
-      const float l_row = l[qi] + swap(qi, nk_all, l[qi]);
-      ok = __all_sync(0xffffffffu, ok && nk_all > 0 &&
-                                       mbar_wait(&ctl.pv_done[qi], (nk_all - 1) & 1, wc, 0x3a));
-      uint8_t* ybuf = q_s + qi * kTileB + half * kHalf;  // Q'_i is no longer read
-      const uint8_t* gbuf = k_s + qi * kTileB + half * kHalf;
-      const uint32_t tmem_o = tmem + 256 + qi * 128 + half * 64;
-      if (ok) {
+      float rs0, rs1;
+      up2(rs2, rs0, rs1);
+      l = l * corr + (rs0 + rs1);
+      m = m_use;
+      if (any_grow && j >= 1) {
+        // O_i holds the sum over tiles < j (their PV MMAs finished before S_i
+        // of this tile was issued); scale it before the next PV accumulates
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctl.pv_done[qi], (j - 1) & 1, wc, 0x39))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const float inv = 1.f / l_row;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tmem_o + lane_base + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {  // 8 columns per 16-byte chunk
-            const int ch = c * 4 + q;
-            const uint32_t off = sw128_off(r, ch);
-            uint32_t gw[4] = {0, 0, 0, 0};
-            if (kGate) {
-              const uint4 gr = *reinterpret_cast<const uint4*>(gbuf + off);
-              gw[0] = gr.x; gw[1] = gr.y; gw[2] = gr.z; gw[3] = gr.w;
-            }
-            uint32_t out[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float y0 = __uint_as_float(o[q * 8 + 2 * i]) * inv;
-              float y1 = __uint_as_float(o[q * 8 + 2 * i + 1]) * inv;
-              if (kGate) {
-                const float2 gg = bf2_to_f2(gw[i]);
-                y0 *= sigmoid_fast(gg.x);
-                y1 *= sigmoid_fast(gg.y);
-              }
-              out[i] = f2_to_bf2(y0, y1);
-            }
-            *reinterpret_cast<uint4*>(ybuf + off) = make_uint4(out[0], out[1], out[2], out[3]);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+          tmem_st32(tmem_o + lane_base + c * 32, o);
         }
-        fence_proxy_async_smem();
       }
-      mbar_arrive(&ctl.ysync[qi]);
-      ok = mbar_wait(&ctl.ysync[qi], 0, wc, 0x3b) && ok;
-      if (ok && r == 0 && half == 0 && row0 + qi * kRows < N) {  // a tile past N has nothing to store
-        uint8_t* yt = q_s + qi * kTileB;
-        tma_store_3d(&tm_y, yt, h * kD, row0 + qi * kRows, b);
-        tma_store_3d(&tm_y, yt + kHalf, h * kD + 64, row0 + qi * kRows, b);
-        bulk_commit();
-        bulk_wait0();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctl.p_full[qi]);
+    }
+    // ---------------- epilogue: Y = O / l * sigmoid(G)
+    ok = __all_sync(0xffffffffu,
+                    ok && nk_all > 0 && mbar_wait(&ctl.pv_done[qi], (nk_all - 1) & 1, wc, 0x3a));
+    if (kGate) ok = ok && __all_sync(0xffffffffu, mbar_wait(&ctl.g_full, 0, wc, 0x3d));
+    uint8_t* ybuf = q_s + qi * kTileB;  // Q'_i is no longer read
+    const uint8_t* gbuf = k_s + qi * kTileB;
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_base + c * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // 8 columns per 16-byte chunk
+          const int ch = (c & 1) * 4 + q;
+          const uint32_t off = (c >> 1) * kHalf + sw128_off(r, ch);
+          uint32_t gw[4] = {0, 0, 0, 0};
+          if (kGate) {
+            const uint4 gr = *reinterpret_cast<const uint4*>(gbuf + off);
+            gw[0] = gr.x; gw[1] = gr.y; gw[2] = gr.z; gw[3] = gr.w;
+          }
+          uint32_t out[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float y0 = __uint_as_float(o[q * 8 + 2 * i]) * inv;
+            float y1 = __uint_as_float(o[q * 8 + 2 * i + 1]) * inv;
+            if (kGate) {
+              const float2 gg = bf2_to_f2(gw[i]);
+              y0 *= sigmoid_fast(gg.x);
+              y1 *= sigmoid_fast(gg.y);
+            }
+            out[i] = f2_to_bf2(y0, y1);
+          }
+          *reinterpret_cast<uint4*>(ybuf + off) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
       }
+      fence_proxy_async_smem();
+    }
+    mbar_arrive(&ctl.ysync[qi]);
+    ok = mbar_wait(&ctl.ysync[qi], 0, wc, 0x3b) && ok;
+    if (ok && r == 0 && row0 + qi * kRows < N) {  // a tile past N has nothing to store
+      tma_store_3d(&tm_y, ybuf, h * kD, row0 + qi * kRows, b);
+      tma_store_3d(&tm_y, ybuf + kHalf, h * kD + 64, row0 + qi * kRows, b);
+      bulk_commit();
+      bulk_wait0();
     }
   }
   tc_fence_before();

@@ -306,80 +306,37 @@ __global__ void __launch_bounds__(1024)
 //   d alpha_s = dh . v_s,  d l_s = alpha_s (d alpha_s - sum_t alpha_t d alpha_t),
 //   d v_s = alpha_s dh + (d l_s / r_s) w - (d l_s l_s / (C r_s^2)) v_s,
 //   d w = sum over tokens of sum_s (d l_s / r_s) v_s.
-// Each warp takes tokens with a fixed stride; the token's source rows and dh
-// arrive in shared memory by bulk copies into a two-stage ring per warp, so
-// the next token's rows are in flight while this one is reduced and
-// differentiated.  Each lane keeps its columns' share of d w in registers and
-// the warp writes one row of d w partials at the end; attnres_dw_reduce_kernel
-// adds the rows in order, so d w is bit-reproducible.
-__device__ __forceinline__ void bulk_row_load(void* smem_dst, const void* src, uint32_t bytes,
-                                              uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
+// Warp per token with a fixed token-to-warp assignment; the token's source
+// rows stay in registers between the reductions and the gradient pass.  Each
+// warp adds its share of d w to its own shared-memory row; the CTA writes the
+// fixed-order sum of its rows and attnres_dw_reduce_kernel adds the CTA rows
+// in order, so d w is bit-reproducible.
+constexpr int kBwdWarps = 8;
 
 template <int NS, int CH>
-__global__ void __launch_bounds__(128)
-    attnres_bwd_staged_kernel(SourcePtrs src, const __nv_bfloat16* __restrict__ dh,
-                              long long tokens, int C, const float* __restrict__ w, float eps,
-                              SourcePtrs dsrc, float* __restrict__ dw_part, int* status) {
-  extern __shared__ __align__(16) uint8_t ring_raw[];  // [warps][2 stages][NS + 1 rows][C] bf16
-  __shared__ uint64_t full[4][2];
-  __shared__ int abort_flag;
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const size_t row_bytes = (size_t)C * 2;
-  const size_t stage_bytes = (NS + 1) * row_bytes;
-  uint8_t* ring = ring_raw + (size_t)wib * 2 * stage_bytes;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < nw; ++i) {
-      mbar_init(&full[i][0], 1);
-      mbar_init(&full[i][1], 1);
-    }
-    abort_flag = 0;
-    mbar_fence_init();
-  }
-  __syncthreads();
-  const WaitCtx wc{&abort_flag, status};
-  const long long gw = (long long)blockIdx.x * nw + wib;   // this warp's first token
-  const long long stride = (long long)gridDim.x * nw;
-  auto issue = [&](long long tok, int stage) {
-    if (lane == 0) {
-      uint8_t* dst = ring + stage * stage_bytes;
-      mbar_arrive_expect_tx(&full[wib][stage], (uint32_t)stage_bytes);
-#pragma unroll
-      for (int s = 0; s < NS; ++s)
-        bulk_row_load(dst + s * row_bytes,
-                      static_cast<const __nv_bfloat16*>(src.p[s]) + (size_t)tok * C,
-                      (uint32_t)row_bytes, &full[wib][stage]);
-      bulk_row_load(dst + NS * row_bytes, dh + (size_t)tok * C, (uint32_t)row_bytes,
-                    &full[wib][stage]);
-    }
-  };
-  float dwv[CH][8];
-#pragma unroll
-  for (int c = 0; c < CH; ++c)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dwv[c][i] = 0.f;
+__global__ void __launch_bounds__(256)
+    attnres_bwd_kernel(SourcePtrs src, const __nv_bfloat16* __restrict__ dh, long long tokens,
+                       int C, const float* __restrict__ w, float eps, SourcePtrs dsrc,
+                       float* __restrict__ dw_part) {
+  extern __shared__ float dw_rows[];  // [kBwdWarps][C]
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* myrow = dw_rows + (size_t)wib * C;
+  for (int i = lane; i < C; i += 32) myrow[i] = 0.f;
+  __syncwarp();
+  const long long nwarps = (long long)gridDim.x * kBwdWarps;
   const float invC = 1.f / (float)C;
-  long long issued = 0;
-  if (gw < tokens) {
-    issue(gw, 0);
-    issued = 1;
-  }
-  long long k = 0;
-  for (long long tok = gw; tok < tokens; tok += stride, ++k) {
-    const int stage = (int)(k & 1);
-    if (tok + stride < tokens) {  // the other stage held token k - 1, already consumed
-      __syncwarp();
-      issue(tok + stride, stage ^ 1);
-      ++issued;
-    }
-    if (!mbar_wait(&full[wib][stage], (uint32_t)(k >> 1) & 1, wc, 0x61)) break;
-    const uint8_t* st = ring + stage * stage_bytes;
-    const __nv_bfloat16* dhs = reinterpret_cast<const __nv_bfloat16*>(st + NS * row_bytes);
+  for (long long tok = (long long)blockIdx.x * kBwdWarps + wib; tok < tokens; tok += nwarps) {
+    const size_t row = (size_t)tok * C;
+    uint4 x[NS][CH];
+#pragma unroll
+    for (int s = 0; s < NS; ++s)
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = (c * 32 + lane) * 8;
+        x[s][c] = col < C ? *reinterpret_cast<const uint4*>(
+                                static_cast<const __nv_bfloat16*>(src.p[s]) + row + col)
+                          : make_uint4(0, 0, 0, 0);
+      }
     float ss[NS], sw[NS], sd[NS];
 #pragma unroll
     for (int s = 0; s < NS; ++s) ss[s] = sw[s] = sd[s] = 0.f;
@@ -387,17 +344,16 @@ __global__ void __launch_bounds__(128)
     for (int c = 0; c < CH; ++c) {
       const int col = (c * 32 + lane) * 8;
       if (col >= C) continue;
-      const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + col));
-      const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + col + 4));
+      const float4 w0 = *reinterpret_cast<const float4*>(w + col);
+      const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
       const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       float dv[8];
       Vec8<__nv_bfloat16> dhc;
-      dhc.load(dhs + col);
+      dhc.load(dh + row + col);
       dhc.to_float(dv);
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(st + s * row_bytes + (size_t)col * 2);
-        const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
+        const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = bf2_to_f2(u[i]);
@@ -439,50 +395,44 @@ __global__ void __launch_bounds__(128)
       cw[s] = dl / r[s];
       cv[s] = -dl * l[s] * invC / (r[s] * r[s]);
     }
-    const size_t row = (size_t)tok * C;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int col = (c * 32 + lane) * 8;
       if (col >= C) continue;
-      const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + col));
-      const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + col + 4));
+      const float4 w0 = *reinterpret_cast<const float4*>(w + col);
+      const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
       const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       float dv[8];
       Vec8<__nv_bfloat16> dhc;
-      dhc.load(dhs + col);
+      dhc.load(dh + row + col);
       dhc.to_float(dv);
+      float dwv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(st + s * row_bytes + (size_t)col * 2);
-        const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
+        const uint32_t u[4] = {x[s][c].x, x[s][c].y, x[s][c].z, x[s][c].w};
         float g[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = bf2_to_f2(u[i]);
           g[2 * i] = fmaf(cv[s], f.x, fmaf(cw[s], wv[2 * i], a[s] * dv[2 * i]));
           g[2 * i + 1] = fmaf(cv[s], f.y, fmaf(cw[s], wv[2 * i + 1], a[s] * dv[2 * i + 1]));
-          dwv[c][2 * i] = fmaf(cw[s], f.x, dwv[c][2 * i]);
-          dwv[c][2 * i + 1] = fmaf(cw[s], f.y, dwv[c][2 * i + 1]);
+          dwv[2 * i] = fmaf(cw[s], f.x, dwv[2 * i]);
+          dwv[2 * i + 1] = fmaf(cw[s], f.y, dwv[2 * i + 1]);
         }
-        Vec8<__nv_bfloat16>::store(
-            static_cast<__nv_bfloat16*>(const_cast<void*>(dsrc.p[s])) + row + col, g);
+        Vec8<__nv_bfloat16>::store(static_cast<__nv_bfloat16*>(const_cast<void*>(dsrc.p[s])) + row + col, g);
       }
+      float4* acc = reinterpret_cast<float4*>(myrow + col);
+      const float4 a0 = acc[0], a1 = acc[1];
+      acc[0] = make_float4(a0.x + dwv[0], a0.y + dwv[1], a0.z + dwv[2], a0.w + dwv[3]);
+      acc[1] = make_float4(a1.x + dwv[4], a1.y + dwv[5], a1.z + dwv[6], a1.w + dwv[7]);
     }
   }
-  // this warp's share of d w, one row per warp
-  float* myrow = dw_part + (size_t)gw * C;
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float acc = 0.f;
 #pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int col = (c * 32 + lane) * 8;
-    if (col >= C) continue;
-    reinterpret_cast<float4*>(myrow + col)[0] =
-        make_float4(dwv[c][0], dwv[c][1], dwv[c][2], dwv[c][3]);
-    reinterpret_cast<float4*>(myrow + col)[1] =
-        make_float4(dwv[c][4], dwv[c][5], dwv[c][6], dwv[c][7]);
-  }
-  if (abort_flag && lane == 0) {  // copies in flight land before the CTA exits
-    for (long long u = issued > 2 ? issued - 2 : 0; u < issued; ++u)
-      mbar_drain(&full[wib][u & 1], (uint32_t)(u >> 1) & 1);
+    for (int k = 0; k < kBwdWarps; ++k) acc += dw_rows[k * C + c];
+    dw_part[(size_t)blockIdx.x * C + c] = acc;
   }
 }
 
@@ -496,41 +446,30 @@ __global__ void __launch_bounds__(256)
   dw[c] = acc;
 }
 
-// Warps per CTA of the staged backward: two ring stages of S + 1 rows of C
-// bf16 per warp within the shared-memory budget, at most 4 (>= 2 for S <= 4
-// and C <= 4096).
-constexpr size_t kBwdSmemMax = 227 * 1024 - 1024;
-int bwd_warps(int S, int C) {
-  const int w = (int)(kBwdSmemMax / (2 * (size_t)(S + 1) * C * 2));
-  return w > 4 ? 4 : w;
-}
-int bwd_blocks(long long tokens, int warps) {
-  const long long want = (tokens + warps - 1) / warps;
-  return (int)(want < kNumSMs ? (want > 0 ? want : 1) : kNumSMs);  // one CTA per SM
+int attnres_bwd_blocks(long long tokens) {
+  const long long want = (tokens + kBwdWarps - 1) / kBwdWarps;
+  const long long cap = kNumSMs;  // one CTA of 8 warps per SM (registers: ~220 per thread at 3 sources)
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
 template <int NS, int CH>
 void bwd_launch(const SourcePtrs& sp, const void* dh, long long tokens, int C, const float* w,
-                float eps, const SourcePtrs& dsp, float* dw_part, int* rows, cudaStream_t st) {
-  const int warps = bwd_warps(NS, C);
-  const int blocks = bwd_blocks(tokens, warps);
-  const int smem = (int)(warps * 2 * (size_t)(NS + 1) * C * 2);
-  cudaFuncSetAttribute(attnres_bwd_staged_kernel<NS, CH>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  attnres_bwd_staged_kernel<NS, CH><<<blocks, warps * 32, smem, st>>>(
-      sp, static_cast<const __nv_bfloat16*>(dh), tokens, C, w, eps, dsp, dw_part, status_word());
-  *rows = blocks * warps;
+                float eps, const SourcePtrs& dsp, float* dw_part, cudaStream_t st) {
+  const int blocks = attnres_bwd_blocks(tokens);
+  const int smem = kBwdWarps * C * (int)sizeof(float);
+  cudaFuncSetAttribute(attnres_bwd_kernel<NS, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  attnres_bwd_kernel<NS, CH><<<blocks, 256, smem, st>>>(
+      sp, static_cast<const __nv_bfloat16*>(dh), tokens, C, w, eps, dsp, dw_part);
 }
 
 template <int CH>
 void bwd_launch_s(const SourcePtrs& sp, int S, const void* dh, long long tokens, int C,
-                  const float* w, float eps, const SourcePtrs& dsp, float* dw_part, int* rows,
-                  cudaStream_t st) {
+                  const float* w, float eps, const SourcePtrs& dsp, float* dw_part, cudaStream_t st) {
   switch (S) {
-    case 1: bwd_launch<1, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, rows, st); break;
-    case 2: bwd_launch<2, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, rows, st); break;
-    case 3: bwd_launch<3, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, rows, st); break;
-    default: bwd_launch<4, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, rows, st); break;
+    case 1: bwd_launch<1, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+    case 2: bwd_launch<2, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+    case 3: bwd_launch<3, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
+    default: bwd_launch<4, CH>(sp, dh, tokens, C, w, eps, dsp, dw_part, st); break;
   }
 }
 
@@ -609,9 +548,7 @@ sana_status attnres_run(int B, long long N, int C, sana_dtype dt, const void* co
 }
 
 size_t attnres_bwd_ws_bytes(long long tokens, int C) {
-  // one row of d w partials per warp: at most 4 warps per CTA, one CTA per SM
-  const long long rows = tokens + 3 < 4LL * kNumSMs ? tokens + 3 : 4LL * kNumSMs;
-  return align_up((size_t)rows * C * sizeof(float), 256);
+  return align_up((size_t)attnres_bwd_blocks(tokens) * C * sizeof(float), 256);
 }
 
 sana_status attnres_bwd_run(long long tokens, int C, const void* const* sources, int S,
@@ -633,13 +570,12 @@ sana_status attnres_bwd_run(long long tokens, int C, const void* const* sources,
   }
   float* dw_part = static_cast<float*>(ws);
   const int ch = C / 256;
-  int rows = 0;
-  if (ch <= 4) bwd_launch_s<4>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, &rows, st);
-  else if (ch <= 8) bwd_launch_s<8>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, &rows, st);
-  else if (ch <= 12) bwd_launch_s<12>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, &rows, st);
-  else bwd_launch_s<16>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, &rows, st);
-  if (sana_status e = check_launch("attnres_bwd_staged_kernel")) return e;
-  attnres_dw_reduce_kernel<<<(C + 255) / 256, 256, 0, st>>>(dw_part, rows, C, dw);
+  if (ch <= 4) bwd_launch_s<4>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  else if (ch <= 8) bwd_launch_s<8>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  else if (ch <= 12) bwd_launch_s<12>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  else bwd_launch_s<16>(sp, S, dh, tokens, C, w, eps, dsp, dw_part, st);
+  if (sana_status e = check_launch("attnres_bwd_kernel")) return e;
+  attnres_dw_reduce_kernel<<<(C + 255) / 256, 256, 0, st>>>(dw_part, attnres_bwd_blocks(tokens), C, dw);
   return check_launch("attnres_dw_reduce_kernel");
 }
 

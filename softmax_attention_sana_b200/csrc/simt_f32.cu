@@ -163,55 +163,61 @@ __global__ void rope_rotate_kernel(const T* __restrict__ x, RopeDev rope, GridDe
   }
 }
 
-// bf16 form: thread c owns the 16-byte chunk c (four rotary pairs of one
-// head) of every token row its CTA visits, so which axis and local frequency
-// each of its pairs takes is decoded once; a CTA walks token rows with a
-// stride of the grid, four rows per iteration with all four loads issued
-// before the first rotation (full-width, coalesced loads and stores; the
-// tables stay in L1).
-constexpr int kRopeRows = 4;
-__global__ void __launch_bounds__(512)
+// bf16 form: a thread owns one 16-byte chunk position within a head (four
+// rotary pairs) of one token and walks that position through every head of
+// the token, so the token's (cos, sin) for its four pairs are read once and
+// used heads times; 16 threads cover one token's chunk positions (D = 128)
+// and a warp two tokens, each a contiguous 256-byte run per head.  Loads of
+// eight heads are in flight before the first rotation.
+constexpr int kRopeHeadsInFlight = 8;
+__global__ void __launch_bounds__(256)
     rope_rotate_bf16x8_kernel(const uint4* __restrict__ x, RopeDev rope, GridDev g, int D,
                               float mul, uint4* __restrict__ out) {
   const int b = blockIdx.y;
-  const int chunks = g.heads * D / 8;  // per token
+  const int cpd = D / 8;                       // chunk positions per head
+  const int tpb = blockDim.x / cpd;            // tokens per block and pass
+  const int cl = threadIdx.x % cpd, tl = threadIdx.x / cpd;
+  const int chunks = g.heads * cpd;            // per token
   const int hw = g.H * g.W;
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-    const int j0 = (c * 8 % D) / 2;  // first rotary pair of the chunk within its head
-    // per pair: table (0 t, 1 h, 2 w) and column within that axis' table
-    int ax[4], col[4];
+  const int j0 = cl * 4;                       // first rotary pair of the chunk
+  int ax[4], col[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int j = j0 + k;
-      ax[k] = j < rope.n_t ? 0 : (j < rope.n_t + rope.n_h ? 1 : 2);
-      col[k] = ax[k] == 0 ? j : (ax[k] == 1 ? j - rope.n_t : j - rope.n_t - rope.n_h);
+  for (int k = 0; k < 4; ++k) {
+    const int j = j0 + k;
+    ax[k] = j < rope.n_t ? 0 : (j < rope.n_t + rope.n_h ? 1 : 2);
+    col[k] = ax[k] == 0 ? j : (ax[k] == 1 ? j - rope.n_t : j - rope.n_t - rope.n_h);
+  }
+  for (int n = blockIdx.x * tpb + tl; n < g.N; n += gridDim.x * tpb) {
+    float2 cs[4];
+    if (rope.cos_t) {
+      const int t = n / hw, rem = n - t * hw, hh = rem / g.W, ww = rem - hh * g.W;
+      const int tt = g.t_offset + b * g.t_stride + t;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int pos = ax[k] == 0 ? tt : (ax[k] == 1 ? hh : ww);
+        const int np = ax[k] == 0 ? rope.n_t : (ax[k] == 1 ? rope.n_h : rope.n_w);
+        const float* ct = ax[k] == 0 ? rope.cos_t : (ax[k] == 1 ? rope.cos_h : rope.cos_w);
+        const float* st = ax[k] == 0 ? rope.sin_t : (ax[k] == 1 ? rope.sin_h : rope.sin_w);
+        cs[k] = make_float2(__ldg(ct + pos * np + col[k]), __ldg(st + pos * np + col[k]));
+      }
     }
-    for (int n0 = blockIdx.x * kRopeRows; n0 < g.N; n0 += gridDim.x * kRopeRows) {
-      uint4 raw[kRopeRows];
+    const size_t row = ((size_t)b * g.N + n) * chunks + cl;
+    for (int h0 = 0; h0 < g.heads; h0 += kRopeHeadsInFlight) {
+      uint4 raw[kRopeHeadsInFlight];
 #pragma unroll
-      for (int u = 0; u < kRopeRows; ++u)
-        raw[u] = n0 + u < g.N ? x[((size_t)b * g.N + n0 + u) * chunks + c] : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < kRopeHeadsInFlight; ++u)
+        raw[u] = h0 + u < g.heads ? x[row + (size_t)(h0 + u) * cpd] : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int u = 0; u < kRopeRows; ++u) {
-        const int n = n0 + u;
-        if (n >= g.N) break;
+      for (int u = 0; u < kRopeHeadsInFlight; ++u) {
+        if (h0 + u >= g.heads) break;
         uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-        const int t = n / hw, rem = n - t * hw, hh = rem / g.W, ww = rem - hh * g.W;
-        const int tt = g.t_offset + b * g.t_stride + t;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           float2 v = bf2_to_f2(w[k]);
-          if (rope.cos_t) {
-            const int pos = ax[k] == 0 ? tt : (ax[k] == 1 ? hh : ww);
-            const int np = ax[k] == 0 ? rope.n_t : (ax[k] == 1 ? rope.n_h : rope.n_w);
-            const float* ct = ax[k] == 0 ? rope.cos_t : (ax[k] == 1 ? rope.cos_h : rope.cos_w);
-            const float* st = ax[k] == 0 ? rope.sin_t : (ax[k] == 1 ? rope.sin_h : rope.sin_w);
-            const int idx = pos * np + col[k];
-            v = rotate(v.x, v.y, make_float2(__ldg(ct + idx), __ldg(st + idx)));
-          }
+          if (rope.cos_t) v = rotate(v.x, v.y, cs[k]);
           w[k] = f2_to_bf2(v.x * mul, v.y * mul);
         }
-        out[((size_t)b * g.N + n) * chunks + c] = make_uint4(w[0], w[1], w[2], w[3]);
+        out[row + (size_t)(h0 + u) * cpd] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
@@ -364,14 +370,14 @@ sana_status rope_rotate_run(const void* x, bool bf16, const RopeDev* rope, const
   int blocks = (int)((pairs + 255) / 256);
   if (blocks > 4 * kNumSMs * 8) blocks = 4 * kNumSMs * 8;
   if (blocks < 1) blocks = 1;
-  if (bf16 && D % 8 == 0) {
-    const int chunks = g.heads * D / 8;  // per token row
-    const int threads = chunks < 512 ? (chunks + 31) / 32 * 32 : 512;
-    // about 2048 resident threads per SM: enough rows in flight to cover HBM latency
-    long long rows_blocks = ((long long)g.N + kRopeRows - 1) / kRopeRows;
-    const long long cap = (long long)kNumSMs * (2048 / threads) / (B > 0 ? B : 1);
-    if (rows_blocks > cap) rows_blocks = cap > 0 ? cap : 1;
-    rope_rotate_bf16x8_kernel<<<dim3((unsigned)rows_blocks, B), threads, 0, st>>>(
+  if (bf16 && D % 8 == 0 && D <= 256) {
+    const int cpd = D / 8;
+    const int threads = 256 / cpd * cpd;       // whole tokens per block
+    const int tpb = threads / cpd;
+    long long nb = ((long long)g.N + tpb - 1) / tpb;
+    const long long cap = (long long)kNumSMs * 8 / (B > 0 ? B : 1);
+    if (nb > cap) nb = cap > 0 ? cap : 1;
+    rope_rotate_bf16x8_kernel<<<dim3((unsigned)nb, B), threads, 0, st>>>(
         static_cast<const uint4*>(x), r, g, D, mul, static_cast<uint4*>(out));
   } else if (bf16)
     rope_rotate_kernel<__nv_bfloat16><<<dim3(blocks, B), 256, 0, st>>>(
