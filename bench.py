@@ -370,14 +370,14 @@ def components(sana, args):
         xq, xs = sana.mx_quantize(A)
         ws_mx = torch.empty(sana._lib.lib.sana_mx_linear_workspace_size(WL.N, WL.C),
                             dtype=torch.uint8, device="cuda")
-        f = lambda: sana.mx_linear(A, wq, wsc, 4 * WL.C, out=Yq, ws=ws_mx)
-        for _ in range(3):
-            f()
-        ms = time_loop(f, 10)
         g = lambda: sana.mx_gemm(xq, xs, wq, wsc, 4 * WL.C, out=Yq)
         for _ in range(3):
             g()
         ms_g = time_loop(g, 10)
+        f = lambda: sana.mx_linear(A, wq, wsc, 4 * WL.C, out=Yq, ws=ws_mx)
+        for _ in range(3):
+            f()
+        ms = time_loop(f, 10)
         q = lambda: sana.mx_quantize(A)
         ms_q = time_loop(q, 10)
         flops = 2 * WL.N * 4 * WL.C * WL.C
@@ -462,9 +462,11 @@ def components(sana, args):
         grid = (WL.T, WL.H, WL.W)
         rope = sana.Rope(WL.T, WL.H, WL.W, WL.rope_split)
         keep = (sana.anchor_tile_count(WL.N) + 3) // 4
-        for name, layers, attnres, ffn, kt in (("stack_720p_group4", 4, False, 0, 0),
-                                                ("stack_720p_group4_sparse25", 4, False, 0, keep),
-                                                ("stack_720p_attnres16", 16, True, 3, 0)):
+        for name, layers, attnres, ffn, kt, mx in (
+                ("stack_720p_group4", 4, False, 0, 0, False),
+                ("stack_720p_group4_sparse25", 4, False, 0, keep, False),
+                ("stack_720p_attnres16", 16, True, 3, 0, False),
+                ("stack_720p_attnres16_mx", 16, True, 3, 0, True)):
             gen = torch.Generator(device="cuda")
             gen.manual_seed(5000 + layers)
             rn = lambda *sh, sc=1.0: (torch.randn(sh, generator=gen, device="cuda") * sc).to(
@@ -479,7 +481,9 @@ def components(sana, args):
                 ws_l.append(d)
             w_attn, w_ffn = (t.cuda() for t in si.router_queries(5, WL.C))
             cfg = sana.stack_config(layers, block_span=8, use_attnres=attnres, ffn_mult=ffn,
-                                    anchor_keep_tiles=kt)
+                                    anchor_keep_tiles=kt, mx_projections=mx)
+            if mx:  # MXFP4 weights quantised once, outside the timing
+                ws_l = sana.mx_quantize_stack_weights(ws_l)
             y = torch.empty_like(x)
             f = lambda: sana.hybrid_stack_fwd(x, ws_l, w_attn, w_ffn, rope, grid, WL.heads, cfg, out=y)
             f()
@@ -499,6 +503,9 @@ def components(sana, args):
                          "timing": "2 calls after 1 warm-up, CUDA events"}
             if kt:
                 out[name]["anchor_keep_tiles"] = kt
+            if mx:
+                out[name]["projections"] = ("MXFP8 activations x MXFP4 weights (flops counted as "
+                                            "for the bf16 stack)")
             del x, ws_l, y
     return out
 

@@ -399,6 +399,11 @@ typedef struct {
   int anchor_keep_tiles; /* 0: dense anchors; k > 0: block-sparse anchors keeping
                             the k highest-scoring 128-key tiles per 256-query
                             block (sana_softmax_anchor_sparse_fwd's selection) */
+  int mx_projections;    /* 0: bf16 projections; 1: every projection (QKVG, O, FFN
+                            up and down) is the MX projection -- activations
+                            quantised to MXFP8 on the fly, MXFP4 weights from the
+                            mx_* arrays of sana_stack_weights (the deployment of
+                            [SV2] Experiments; attention stays bf16) */
 } sana_stack_config;
 
 typedef struct {
@@ -408,6 +413,17 @@ typedef struct {
   const void* const* w_down; /* [layers] of (C, ffn_mult*C), or NULL */
   const float* w_attn;       /* device fp32 (C): shared attention router query */
   const float* w_ffn;        /* device fp32 (C): shared FFN router query */
+  /* With cfg->mx_projections: per layer, each weight as sana_mx_quantize writes
+     it with fp4 = 1 (E2M1 codes, 32-byte aligned, and scale atoms); the bf16
+     arrays above are then not read and may be NULL. */
+  const void* const* mx_qkvg;
+  const void* const* mx_qkvg_scales;
+  const void* const* mx_o;
+  const void* const* mx_o_scales;
+  const void* const* mx_up;
+  const void* const* mx_up_scales;
+  const void* const* mx_down;
+  const void* const* mx_down_scales;
 } sana_stack_weights;
 
 SANA_API size_t sana_hybrid_stack_workspace_size(const sana_shape* shape, const sana_stack_config* cfg);

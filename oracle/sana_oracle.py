@@ -524,9 +524,20 @@ def is_anchor_layer(l, ratio=4):
     return l % ratio == ratio - 1
 
 
-def _attention_sublayer(xh, Wl, grid, rope_split, heads, eps, anchor, anchor_keep=0):
+def _project(x, W, mx=False):
+    """x W^T: exact, or the MX projection Q8(x) Q4(W)^T ([SV2] Experiments:
+    the deployment quantises the linear GEMMs, MXFP8 activations and MXFP4
+    weights) through mx_linear, blocked along the contraction axis."""
+    W = np.asarray(W, np.float64)
+    if not mx:
+        return x @ W.T
+    lead = x.shape[:-1]
+    return mx_linear(np.asarray(x, np.float64).reshape(-1, x.shape[-1]), W).reshape(*lead, -1)
+
+
+def _attention_sublayer(xh, Wl, grid, rope_split, heads, eps, anchor, anchor_keep=0, mx=False):
     C = xh.shape[-1]
-    qkvg = xh @ np.asarray(Wl['qkvg'], np.float64).T
+    qkvg = _project(xh, Wl['qkvg'], mx)
     q, k, v, g = (qkvg[..., i * C:(i + 1) * C] for i in range(4))
     if anchor and anchor_keep > 0:
         tiles = anchor_block_select(anchor_block_scores(q, k, grid, rope_split, heads), anchor_keep)
@@ -535,17 +546,17 @@ def _attention_sublayer(xh, Wl, grid, rope_split, heads, eps, anchor, anchor_kee
         a = softmax_anchor(q, k, v, grid, rope_split, heads, gate=g)
     else:
         a, _, _ = linattn_bidirectional(q, k, v, grid, rope_split, heads, gate=g, eps=eps)
-    return a @ np.asarray(Wl['o'], np.float64).T
+    return _project(a, Wl['o'], mx)
 
 
-def _ffn_sublayer(xh, Wl):
-    u = silu(xh @ np.asarray(Wl['up'], np.float64).T)
-    return u @ np.asarray(Wl['down'], np.float64).T
+def _ffn_sublayer(xh, Wl, mx=False):
+    u = silu(_project(xh, Wl['up'], mx))
+    return _project(u, Wl['down'], mx)
 
 
 def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
                  block_span=8, ratio=4, use_attnres=True, ffn=True, eps=EPS,
-                 rms_eps=RMS_EPS, anchor_keep=0):
+                 rms_eps=RMS_EPS, anchor_keep=0, mx=False):
     """Forward of the hybrid stack.
 
     With AttnRes: every sublayer reads h = route(V_l) over [embedding,
@@ -554,15 +565,17 @@ def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
     frozen as a block summary.  The result is the representation a next layer
     would read: route(V, w_attn) over the final source set.
     Without AttnRes: plain pre-norm residual x += sublayer(RMSNorm(x)).
-    anchor_keep > 0: the anchors are block-sparse (anchor_block_select's tiles)."""
+    anchor_keep > 0: the anchors are block-sparse (anchor_block_select's tiles).
+    mx: every projection (QKVG, O, FFN up and down) is the MX projection
+    (mx_linear); attention, routes and norms stay exact."""
     x = np.asarray(x, np.float64)
     if not use_attnres:
         for l in range(layers):
             Wl = weights[l]
             x = x + _attention_sublayer(rmsnorm(x, rms_eps), Wl, grid, rope_split,
-                                        heads, eps, is_anchor_layer(l, ratio), anchor_keep)
+                                        heads, eps, is_anchor_layer(l, ratio), anchor_keep, mx)
             if ffn:
-                x = x + _ffn_sublayer(rmsnorm(x, rms_eps), Wl)
+                x = x + _ffn_sublayer(rmsnorm(x, rms_eps), Wl, mx)
         return x
     summaries = []
     partial = None
@@ -574,11 +587,11 @@ def hybrid_stack(x, weights, w_attn, w_ffn, grid, rope_split, heads, layers,
         Wl = weights[l]
         h, _ = attnres_route(sources(), w_attn, rms_eps)
         out = _attention_sublayer(rmsnorm(h, rms_eps), Wl, grid, rope_split, heads,
-                                  eps, is_anchor_layer(l, ratio), anchor_keep)
+                                  eps, is_anchor_layer(l, ratio), anchor_keep, mx)
         partial = out if partial is None else partial + out
         if ffn:
             h, _ = attnres_route(sources(), w_ffn, rms_eps)
-            partial = partial + _ffn_sublayer(rmsnorm(h, rms_eps), Wl)
+            partial = partial + _ffn_sublayer(rmsnorm(h, rms_eps), Wl, mx)
         if (l + 1) % block_span == 0:
             summaries.append(partial)
             partial = None

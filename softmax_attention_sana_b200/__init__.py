@@ -10,7 +10,8 @@ from ._lib import (EPI_NONE, EPI_RESIDUAL, EPI_SILU, Rope, SanaError, attnres_ro
                    hybrid_stack_workspace_views, last_error, lib,
                    linattn_apply, linattn_bwd, linattn_block_causal_scan, linattn_block_causal_scan_workspace_size,
                    linattn_block_causal_step, linattn_fwd, linattn_state,
-                   linattn_workspace_size, mx_gemm, mx_linear, mx_quantize, rmsnorm, rope_apply,
+                   linattn_workspace_size, mx_gemm, mx_linear, mx_quantize, mx_quantize_stack_weights,
+                   rmsnorm, rope_apply,
                    softmax_anchor_rotated_fwd,
                    anchor_tile_count, softmax_anchor_fwd, softmax_anchor_sparse_fwd,
                    softmax_anchor_sparse_workspace_size, stack_config,
@@ -23,7 +24,8 @@ __all__ = [
     "hybrid_stack_workspace_views", "last_error", "lib",
     "linattn_apply", "linattn_bwd", "linattn_block_causal_scan", "linattn_block_causal_scan_workspace_size",
     "linattn_block_causal_step", "linattn_fwd", "linattn_state", "linattn_workspace_size", "rmsnorm",
-    "mx_gemm", "mx_linear", "mx_quantize", "rope_apply", "softmax_anchor_rotated_fwd",
+    "mx_gemm", "mx_linear", "mx_quantize", "mx_quantize_stack_weights", "rope_apply",
+    "softmax_anchor_rotated_fwd",
     "anchor_tile_count", "softmax_anchor_fwd", "softmax_anchor_sparse_fwd",
     "softmax_anchor_sparse_workspace_size", "stack_config",
     "sync_status",

@@ -46,13 +46,18 @@ class RopeStruct(Structure):
 class StackConfig(Structure):
     _fields_ = [("layers", c_int), ("block_span", c_int), ("ratio", c_int), ("use_attnres", c_int),
                 ("ffn_mult", c_int), ("eps", c_float), ("rms_eps", c_float),
-                ("anchor_scale", c_float), ("anchor_keep_tiles", c_int)]
+                ("anchor_scale", c_float), ("anchor_keep_tiles", c_int),
+                ("mx_projections", c_int)]
 
 
 class StackWeights(Structure):
     _fields_ = [("w_qkvg", POINTER(c_void_p)), ("w_o", POINTER(c_void_p)),
                 ("w_up", POINTER(c_void_p)), ("w_down", POINTER(c_void_p)),
-                ("w_attn", c_void_p), ("w_ffn", c_void_p)]
+                ("w_attn", c_void_p), ("w_ffn", c_void_p),
+                ("mx_qkvg", POINTER(c_void_p)), ("mx_qkvg_scales", POINTER(c_void_p)),
+                ("mx_o", POINTER(c_void_p)), ("mx_o_scales", POINTER(c_void_p)),
+                ("mx_up", POINTER(c_void_p)), ("mx_up_scales", POINTER(c_void_p)),
+                ("mx_down", POINTER(c_void_p)), ("mx_down_scales", POINTER(c_void_p))]
 
 
 class StackWsLayout(Structure):
@@ -489,9 +494,24 @@ def gemm_bf16(A, W, out=None, epilogue=EPI_NONE):
 # ---------------------------------------------------------------- stack
 
 def stack_config(layers, block_span=8, ratio=4, use_attnres=True, ffn_mult=3, eps=1e-6,
-                 rms_eps=1e-6, anchor_scale=0.0, anchor_keep_tiles=0) -> StackConfig:
+                 rms_eps=1e-6, anchor_scale=0.0, anchor_keep_tiles=0,
+                 mx_projections=False) -> StackConfig:
     return StackConfig(layers, block_span, ratio, int(bool(use_attnres)), ffn_mult, eps, rms_eps,
-                       anchor_scale, anchor_keep_tiles)
+                       anchor_scale, anchor_keep_tiles, int(bool(mx_projections)))
+
+
+def mx_quantize_stack_weights(weights):
+    """Per-layer weight dicts with the MX form of every projection weight added
+    (keys '<name>_mxq' codes and '<name>_mxs' scales), as the stack reads them
+    with mx_projections on."""
+    out = []
+    for d in weights:
+        e = dict(d)
+        for key in ("qkvg", "o", "up", "down"):
+            if key in d:
+                e[key + "_mxq"], e[key + "_mxs"] = mx_quantize(d[key], fp4=True)
+        out.append(e)
+    return out
 
 
 def hybrid_stack_fwd(x, weights, w_attn, w_ffn, rope: Rope, grid, heads, cfg: StackConfig,
@@ -502,16 +522,20 @@ def hybrid_stack_fwd(x, weights, w_attn, w_ffn, rope: Rope, grid, heads, cfg: St
     L = cfg.layers
 
     def arr(key):
-        if cfg.ffn_mult == 0 and key in ("up", "down"):
+        if cfg.ffn_mult == 0 and key.split("_")[0] in ("up", "down"):
+            return None
+        if any(key not in weights[l] for l in range(L)):
             return None
         return (c_void_p * L)(*[weights[l][key].data_ptr() for l in range(L)])
 
-    keep = {k: arr(k) for k in ("qkvg", "o", "up", "down")}
+    names = ("qkvg", "o", "up", "down")
+    keep = {k: arr(k) for k in names + tuple(n + sfx for n in names for sfx in ("_mxq", "_mxs"))}
+    p = lambda a: None if a is None else ctypes.cast(a, POINTER(c_void_p))
     sw = StackWeights(
-        ctypes.cast(keep["qkvg"], POINTER(c_void_p)), ctypes.cast(keep["o"], POINTER(c_void_p)),
-        None if keep["up"] is None else ctypes.cast(keep["up"], POINTER(c_void_p)),
-        None if keep["down"] is None else ctypes.cast(keep["down"], POINTER(c_void_p)),
-        None if w_attn is None else w_attn.data_ptr(), None if w_ffn is None else w_ffn.data_ptr())
+        p(keep["qkvg"]), p(keep["o"]), p(keep["up"]), p(keep["down"]),
+        None if w_attn is None else w_attn.data_ptr(), None if w_ffn is None else w_ffn.data_ptr(),
+        p(keep["qkvg_mxq"]), p(keep["qkvg_mxs"]), p(keep["o_mxq"]), p(keep["o_mxs"]),
+        p(keep["up_mxq"]), p(keep["up_mxs"]), p(keep["down_mxq"]), p(keep["down_mxs"]))
     if out is None:
         out = torch.empty_like(x)
     if ws is None:

@@ -306,33 +306,43 @@ __global__ void __launch_bounds__(1024)
 //   d alpha_s = dh . v_s,  d l_s = alpha_s (d alpha_s - sum_t alpha_t d alpha_t),
 //   d v_s = alpha_s dh + (d l_s / r_s) w - (d l_s l_s / (C r_s^2)) v_s,
 //   d w = sum over tokens of sum_s (d l_s / r_s) v_s.
-// Warp per token with a fixed token-to-warp assignment; the token's source
-// rows stay in registers between the reductions and the gradient pass.  Each
+// Two warps per token (a warp pair of the CTA), each holding one half of the
+// token's columns of every source in registers between the reductions and
+// the gradient pass; the pair adds its partial sums (sum v^2, w.v, dh.v per
+// source) through shared memory behind a named barrier of the pair, half 0's
+// first (fixed order).  Halving the registers per thread puts two CTAs, 16
+// warps, on an SM: twice the loads in flight of one warp per token.  Each
 // warp adds its share of d w to its own shared-memory row; the CTA writes the
 // fixed-order sum of its rows and attnres_dw_reduce_kernel adds the CTA rows
 // in order, so d w is bit-reproducible.
-constexpr int kBwdWarps = 8;
+constexpr int kBwdWarps = 8;   // 4 pairs
+constexpr int kBwdPairs = 4;
 
 template <int NS, int CH>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
     attnres_bwd_kernel(SourcePtrs src, const __nv_bfloat16* __restrict__ dh, long long tokens,
                        int C, const float* __restrict__ w, float eps, SourcePtrs dsrc,
                        float* __restrict__ dw_part) {
   extern __shared__ float dw_rows[];  // [kBwdWarps][C]
+  __shared__ float xch[2][kBwdPairs][2][3 * NS];
+  constexpr int CHH = (CH + 1) / 2;   // chunks of 256 columns per half
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int pair = wib & (kBwdPairs - 1), half = wib / kBwdPairs;
   float* myrow = dw_rows + (size_t)wib * C;
   for (int i = lane; i < C; i += 32) myrow[i] = 0.f;
   __syncwarp();
-  const long long nwarps = (long long)gridDim.x * kBwdWarps;
+  const long long npairs = (long long)gridDim.x * kBwdPairs;
   const float invC = 1.f / (float)C;
-  for (long long tok = (long long)blockIdx.x * kBwdWarps + wib; tok < tokens; tok += nwarps) {
+  int par = 0;
+  for (long long tok = (long long)blockIdx.x * kBwdPairs + pair; tok < tokens;
+       tok += npairs, par ^= 1) {
     const size_t row = (size_t)tok * C;
-    uint4 x[NS][CH];
+    uint4 x[NS][CHH];
 #pragma unroll
     for (int s = 0; s < NS; ++s)
 #pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        const int col = (c * 32 + lane) * 8;
+      for (int c = 0; c < CHH; ++c) {
+        const int col = ((half * CHH + c) * 32 + lane) * 8;
         x[s][c] = col < C ? *reinterpret_cast<const uint4*>(
                                 static_cast<const __nv_bfloat16*>(src.p[s]) + row + col)
                           : make_uint4(0, 0, 0, 0);
@@ -341,8 +351,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int s = 0; s < NS; ++s) ss[s] = sw[s] = sd[s] = 0.f;
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int col = (c * 32 + lane) * 8;
+    for (int c = 0; c < CHH; ++c) {
+      const int col = ((half * CHH + c) * 32 + lane) * 8;
       if (col >= C) continue;
       const float4 w0 = *reinterpret_cast<const float4*>(w + col);
       const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
@@ -363,7 +373,6 @@ __global__ void __launch_bounds__(256)
         }
       }
     }
-    float a[NS], l[NS], r[NS], m = -INFINITY;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
 #pragma unroll
@@ -372,6 +381,26 @@ __global__ void __launch_bounds__(256)
         sw[s] += __shfl_xor_sync(0xffffffffu, sw[s], o);
         sd[s] += __shfl_xor_sync(0xffffffffu, sd[s], o);
       }
+    }
+    // the pair's halves meet: half 0's partials plus half 1's, in that order
+    if (lane == 0) {
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        xch[par][pair][half][3 * s] = ss[s];
+        xch[par][pair][half][3 * s + 1] = sw[s];
+        xch[par][pair][half][3 * s + 2] = sd[s];
+      }
+    }
+    named_bar_sync(1 + pair, 64);
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      ss[s] = xch[par][pair][0][3 * s] + xch[par][pair][1][3 * s];
+      sw[s] = xch[par][pair][0][3 * s + 1] + xch[par][pair][1][3 * s + 1];
+      sd[s] = xch[par][pair][0][3 * s + 2] + xch[par][pair][1][3 * s + 2];
+    }
+    float a[NS], l[NS], r[NS], m = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
       r[s] = sqrtf(ss[s] * invC + eps);
       l[s] = sw[s] / r[s];
       m = fmaxf(m, l[s]);
@@ -396,8 +425,8 @@ __global__ void __launch_bounds__(256)
       cv[s] = -dl * l[s] * invC / (r[s] * r[s]);
     }
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int col = (c * 32 + lane) * 8;
+    for (int c = 0; c < CHH; ++c) {
+      const int col = ((half * CHH + c) * 32 + lane) * 8;
       if (col >= C) continue;
       const float4 w0 = *reinterpret_cast<const float4*>(w + col);
       const float4 w1 = *reinterpret_cast<const float4*>(w + col + 4);
@@ -447,8 +476,8 @@ __global__ void __launch_bounds__(256)
 }
 
 int attnres_bwd_blocks(long long tokens) {
-  const long long want = (tokens + kBwdWarps - 1) / kBwdWarps;
-  const long long cap = kNumSMs;  // one CTA of 8 warps per SM (registers: ~220 per thread at 3 sources)
+  const long long want = (tokens + kBwdPairs - 1) / kBwdPairs;
+  const long long cap = 2LL * kNumSMs;  // two CTAs of 8 warps (4 token pairs) per SM
   return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 

@@ -20,12 +20,13 @@
 //     layout tcgen05.cp.32x128b.warpx4 copies to TMEM so that each row's four
 //     block scales form one 32-bit TMEM word.
 //
-// GEMM: persistent, 128 x 128 output tiles, a TMA producer warp fills a
-// 6-stage ring of (A 128x128 E4M3, B 128x128 E2M1 unpacked to the 8-bit
-// shared-memory footprint by the 16U4_ALIGN16B tensor map, both scale atoms
-// by bulk copy); one thread copies the scale atoms to TMEM and issues
-// tcgen05.mma kind::mxf8f6f4 (block scale 1X, K = 32 per instruction) into
-// one of two TMEM accumulators while four epilogue warps drain the other.
+// GEMM: persistent, 128 x 256 output tiles (128 x 128 when N is not a
+// multiple of 256); a TMA producer warp fills a ring of stages of (A 128 x 128
+// E4M3, B BN x 128 E2M1 unpacked to the 8-bit shared-memory footprint by the
+// 16U4_ALIGN16B tensor map, the scale atoms by bulk copy); one thread copies
+// the scale atoms to TMEM and issues tcgen05.mma kind::mxf8f6f4 (block scale
+// 1X, K = 32 per instruction); epilogue warps drain the accumulator (the
+// 128-wide form keeps two, so its epilogue overlaps the next tile).
 #include <cuda.h>
 
 #include "sana_common.cuh"
@@ -34,16 +35,29 @@
 namespace sana {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 128;  // BK in elements
-constexpr int kStages = 6;
-constexpr int kABytes = BM * BK;             // E4M3: 16 KB
-constexpr int kBBytes = BN * BK;             // E2M1 in the 8-bit footprint: 16 KB
-constexpr int kSFBytes = 512;                // one scale atom
-constexpr int kStageBytes = kABytes + kBBytes + 2 * kSFBytes;
-// bytes the stage's copies deliver: B arrives as packed nibbles (8 KB)
-constexpr uint32_t kStageTx = kABytes + BN * BK / 2 + 2 * kSFBytes;
-constexpr int kThreads = 192;  // producer, MMA, 4 epilogue warps
-constexpr int kSfCol = 256;    // TMEM column of the scale slots (after 2 accumulators)
+constexpr int BM = 128, BK = 128;  // BK in elements
+constexpr int kABytes = BM * BK;   // E4M3: 16 KB
+constexpr int kSFBytes = 512;      // one scale atom
+constexpr int kSfCol = 256;        // TMEM column of the scale slots (after the accumulators)
+
+// Two tile widths.  BN = 256 (N a multiple of 256) doubles the work of every
+// block-scaled MMA instruction; its 256-column accumulator leaves no room for
+// a second one next to the scale slots, so eight epilogue warps drain it.
+// BN = 128 keeps two accumulators (the epilogue overlaps the next tile).
+template <int BN>
+struct MxCfg {
+  static constexpr int kStages = BN == 128 ? 6 : 4;
+  static constexpr int kAccBufs = BN == 128 ? 2 : 1;
+  static constexpr int kEpiWarps = BN / 32;                   // lane quarter x 128 columns
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;        // producer, MMA, epilogue
+  static constexpr int kBBytes = BN * BK;                     // E2M1 in the 8-bit footprint
+  static constexpr int kSFB = BN / 128 * kSFBytes;            // scale atoms of the B tile
+  static constexpr int kStageBytes = kABytes + kBBytes + kSFBytes + kSFB;
+  // bytes the stage's copies deliver: B arrives as packed nibbles
+  static constexpr uint32_t kStageTx = kABytes + BN * BK / 2 + kSFBytes + kSFB;
+  static constexpr int kSlotCols = 16;                        // A: 4 columns, B: 4 per atom
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes;
+};
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -190,19 +204,30 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
       : "memory");
 }
 
+// Output columns, optionally split into equal parts written to separate
+// tensors (the Q, K, V, G projection).
+struct MxOut {
+  __nv_bfloat16* part[4];
+  int part_cols;  // columns per part (== N when not split), a multiple of BN
+  long long ldo;  // row stride of each part in elements
+};
+
 struct MxCtl {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[6], empty[6];
   uint64_t tfull[2], tempty[2];
   uint64_t drain;  // teardown after an abort: all issued tcgen05 ops finished
   uint32_t tmem;
   int abort_flag;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN>
+__global__ void __launch_bounds__(MxCfg<BN>::kThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, long long M,
-                   int N, int K, __nv_bfloat16* __restrict__ out, long long ldo, int epilogue,
-                   int* status) {
+                   int N, int K, MxOut out, int epilogue, int* status) {
+  using Cfg = MxCfg<BN>;
+  constexpr int kStages = Cfg::kStages, kAccBufs = Cfg::kAccBufs;
+  constexpr int kBBytes = Cfg::kBBytes, kStageBytes = Cfg::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   __shared__ MxCtl ctl;
   uint8_t* smem = align1024(smem_raw);
@@ -218,9 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&ctl.tfull[i], 1);
-      mbar_init(&ctl.tempty[i], 128);
+      mbar_init(&ctl.tempty[i], 32 * Cfg::kEpiWarps);
     }
     mbar_init(&ctl.drain, 1);
     ctl.abort_flag = 0;
@@ -253,13 +278,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&ctl.full[s], kStageTx);
+          mbar_arrive_expect_tx(&ctl.full[s], Cfg::kStageTx);
           tma_load_2d(st, &tm_a, &ctl.full[s], kb * BK, (int)(mt * BM));
           tma_load_2d(st + kABytes, &tm_b, &ctl.full[s], kb * BK, nt * BN);
           bulk_load(st + kABytes + kBBytes, sfa + ((size_t)mt * kblocks + kb) * kSFBytes, kSFBytes,
                     &ctl.full[s]);
-          bulk_load(st + kABytes + kBBytes + kSFBytes,
-                    sfb + ((size_t)nt * kblocks + kb) * kSFBytes, kSFBytes, &ctl.full[s]);
+#pragma unroll
+          for (int a = 0; a < BN / 128; ++a)  // B's scale atoms: 128 rows each
+            bulk_load(st + kABytes + kBBytes + (1 + a) * kSFBytes,
+                      sfb + ((size_t)(nt * (BN / 128) + a) * kblocks + kb) * kSFBytes, kSFBytes,
+                      &ctl.full[s]);
         }
       }
       if (!ok)  // loads in flight land before the CTA exits
@@ -276,8 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int local = 0;
       bool ok = true;
       for (long long t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
-        const int tb = local & 1;
-        if (local >= 2 && !mbar_wait(&ctl.tempty[tb], ((local >> 1) - 1) & 1, wc, 0x52)) break;
+        const int tb = local % kAccBufs;
+        if (local >= kAccBufs &&
+            !mbar_wait(&ctl.tempty[tb], ((local / kAccBufs) - 1) & 1, wc, 0x52))
+          break;
         tc_fence_after();
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = (int)(it % kStages);
@@ -286,10 +316,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          // four scale slots of 8 columns (A: 4, B: 4), rotated per K-block
-          const uint32_t slot = tmem + kSfCol + (uint32_t)(it & 3) * 8;
-          tmem_cp_sf(slot, desc_advance(dsf0, s * kStageBytes));
-          tmem_cp_sf(slot + 4, desc_advance(dsf0, s * kStageBytes + kSFBytes));
+          // four scale slots (A: 4 columns, B: 4 per atom), rotated per K-block
+          const uint32_t slot = tmem + kSfCol + (uint32_t)(it & 3) * Cfg::kSlotCols;
+#pragma unroll
+          for (int a = 0; a <= BN / 128; ++a)
+            tmem_cp_sf(slot + 4 * a, desc_advance(dsf0, s * kStageBytes + a * kSFBytes));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             // the scale-factor id (byte of the TMEM word) is also carried in
@@ -305,21 +336,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps 2..5: TMEM lane quarter = warp % 4
+    // ---------------- epilogue warps: TMEM lane quarter = warp % 4, and
+    // 128 columns per warp of the same quarter
     const int q4 = warp & 3, r = q4 * 32 + lane;
+    const int cbase = ((warp - 2) >> 2) * 128;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     int local = 0;
     for (long long t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
-      const int tb = local & 1;
-      const bool okw = __all_sync(0xffffffffu, mbar_wait(&ctl.tfull[tb], (local >> 1) & 1, wc, 0x54));
+      const int tb = local % kAccBufs;
+      const bool okw = __all_sync(
+          0xffffffffu, mbar_wait(&ctl.tfull[tb], (local / kAccBufs) & 1, wc, 0x54));
       tc_fence_after();
       const long long row = (t / tiles_n) * BM + r;
-      const int n0 = (int)(t % tiles_n) * BN;
-      __nv_bfloat16* orow = out + row * ldo + n0;
+      const int nt0 = (int)(t % tiles_n) * BN;
+      const int part = nt0 / out.part_cols;
+      __nv_bfloat16* orow = out.part[part] + row * out.ldo + (nt0 - part * out.part_cols) + cbase;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
-        if (okw) tmem_ld32(tmem + lane_base + tb * BN + c * 32, v);
+        if (okw) tmem_ld32(tmem + lane_base + tb * BN + cbase + c * 32, v);
         tmem_ld_wait();
         if (!okw || row >= M) continue;
         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -363,8 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-constexpr size_t kMxSmem = 1024 + kStages * kStageBytes;
-
 }  // namespace
 
 size_t mx_scale_bytes(long long rows, int K) {
@@ -389,10 +422,10 @@ sana_status mx_quantize_run(const void* x, long long rows, int K, bool fp4, void
   return check_launch("mx_quant_kernel");
 }
 
-sana_status mx_gemm_run(long long M, int N, int K, const void* xq, const void* xsf,
-                        const void* wq, const void* wsf, void* out, long long ldo, int epilogue,
-                        cudaStream_t st) {
-  if (M == 0) return SANA_OK;
+template <int BN>
+sana_status mx_gemm_launch(long long M, int N, int K, const void* xq, const void* xsf,
+                           const void* wq, const void* wsf, const MxOut& out, int epilogue,
+                           cudaStream_t st) {
   CUtensorMap ta, tb;
   if (!make_tmap_2d_typed(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K, (uint64_t)M,
                           (uint64_t)K, BK, BM) ||
@@ -403,15 +436,40 @@ sana_status mx_gemm_run(long long M, int N, int K, const void* xq, const void* x
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr[dev]) {
-    cudaFuncSetAttribute(mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMxSmem);
+    cudaFuncSetAttribute(mx_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)MxCfg<BN>::kSmem);
     attr[dev] = true;
   }
   const long long tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < kNumSMs ? tiles : kNumSMs);
-  mx_gemm_kernel<<<grid, kThreads, kMxSmem, st>>>(
-      ta, tb, static_cast<const uint8_t*>(xsf), static_cast<const uint8_t*>(wsf), M, N, K,
-      static_cast<__nv_bfloat16*>(out), ldo, epilogue, status_word());
+  mx_gemm_kernel<BN><<<grid, MxCfg<BN>::kThreads, MxCfg<BN>::kSmem, st>>>(
+      ta, tb, static_cast<const uint8_t*>(xsf), static_cast<const uint8_t*>(wsf), M, N, K, out,
+      epilogue, status_word());
   return check_launch("mx_gemm_kernel");
+}
+
+sana_status mx_gemm_run_parts(long long M, int N, int K, const void* xq, const void* xsf,
+                              const void* wq, const void* wsf, void* const* outs, int nparts,
+                              long long ldo, int epilogue, cudaStream_t st) {
+  if (M == 0) return SANA_OK;
+  if (nparts < 1 || nparts > 4 || N % nparts != 0)
+    return fail(SANA_ERR_UNSUPPORTED, "mx gemm: bad output split");
+  MxOut o{};
+  for (int i = 0; i < nparts; ++i) o.part[i] = static_cast<__nv_bfloat16*>(outs[i]);
+  o.part_cols = N / nparts;
+  o.ldo = ldo;
+  // the 256-wide tile when every part is a whole number of them
+  if (N % 256 == 0 && o.part_cols % 256 == 0)
+    return mx_gemm_launch<256>(M, N, K, xq, xsf, wq, wsf, o, epilogue, st);
+  if (o.part_cols % 128 != 0) return fail(SANA_ERR_UNSUPPORTED, "mx gemm: bad output split");
+  return mx_gemm_launch<128>(M, N, K, xq, xsf, wq, wsf, o, epilogue, st);
+}
+
+sana_status mx_gemm_run(long long M, int N, int K, const void* xq, const void* xsf,
+                        const void* wq, const void* wsf, void* out, long long ldo, int epilogue,
+                        cudaStream_t st) {
+  void* outs[1] = {out};
+  return mx_gemm_run_parts(M, N, K, xq, xsf, wq, wsf, outs, 1, ldo, epilogue, st);
 }
 
 }  // namespace sana

@@ -89,15 +89,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
   }
 }
-// The same bounded wait taken by one lane for the whole warp (call with all
-// 32 lanes converged): lane 0 polls, the others wait in the shuffle that
-// hands them the outcome, so a waiting warp issues one poll instead of 32.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w,
-                                               int where, uint64_t limit_ns = kWaitLimitNs) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w, where, limit_ns);
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-}
 // Bounded wait that ignores the abort flag (teardown after an abort).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();

@@ -203,5 +203,9 @@ sana_status mx_quantize_run(const void* x, long long rows, int K, bool fp4, void
 sana_status mx_gemm_run(long long M, int N, int K, const void* xq, const void* xsf,
                         const void* wq, const void* wsf, void* out, long long ldo, int epilogue,
                         cudaStream_t st);
+// The same with the output columns split into nparts equal tensors.
+sana_status mx_gemm_run_parts(long long M, int N, int K, const void* xq, const void* xsf,
+                              const void* wq, const void* wsf, void* const* outs, int nparts,
+                              long long ldo, int epilogue, cudaStream_t st);
 
 }  // namespace sana

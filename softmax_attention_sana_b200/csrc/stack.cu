@@ -39,6 +39,7 @@ struct StackWs {
   void* attn_ws;
   size_t attn_ws_bytes;
   int* tiles;  // kept key tiles of the sparse anchors
+  uint8_t *mxq, *mxs;  // quantised activations of the MX projections (codes, scales)
   size_t bytes;
 };
 
@@ -66,6 +67,11 @@ StackWs carve_stack(const sana_shape& s, const sana_stack_config& c, void* ws) {
     const size_t ntiles = (tok / s.B + 127) / 128;
     w.tiles = cv.take<int>((size_t)s.B * s.heads * ((ntiles + 1) / 2) * c.anchor_keep_tiles);
   }
+  if (c.mx_projections) {
+    const size_t kmax = c.ffn_mult > 1 ? C * c.ffn_mult : C;  // widest contraction
+    w.mxq = cv.take<uint8_t>(tok * kmax);
+    w.mxs = cv.take<uint8_t>(mx_scale_bytes((long long)tok, (int)kmax));
+  }
   w.bytes = align_up(cv.used, 256);
   return w;
 }
@@ -80,6 +86,8 @@ sana_status check_cfg(const sana_shape* s, const sana_stack_config* c) {
   if (c->layers < 1 || c->ratio < 1 || c->ffn_mult < 0 || c->ffn_mult > 8 ||
       (c->use_attnres && c->block_span < 1))
     return fail(SANA_ERR_INVALID_ARG, "stack: bad config");
+  if (c->mx_projections != 0 && c->mx_projections != 1)
+    return fail(SANA_ERR_INVALID_ARG, "stack: mx_projections must be 0 or 1");
   if (c->use_attnres && 1 + (c->layers + c->block_span - 1) / c->block_span > 16)
     return fail(SANA_ERR_UNSUPPORTED, "stack: more than 16 AttnRes sources");
   if (!(c->eps >= 0.f) || !(c->rms_eps >= 0.f)) return fail(SANA_ERR_INVALID_ARG, "stack: bad eps");
@@ -129,10 +137,15 @@ extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_sta
                                              const void* x_embed, void* out, void* ws,
                                              size_t ws_bytes, sana_stream_t st) {
   if (sana_status e = check_cfg(s, c)) return e;
-  if (!w || !rope || !x_embed || !out || !w->w_qkvg || !w->w_o)
+  const bool mx = c->mx_projections != 0;
+  if (!w || !rope || !x_embed || !out)
     return fail(SANA_ERR_INVALID_ARG, "stack: NULL argument");
-  if (c->ffn_mult > 0 && (!w->w_up || !w->w_down))
-    return fail(SANA_ERR_INVALID_ARG, "stack: FFN weights are NULL");
+  if (!mx && (!w->w_qkvg || !w->w_o || (c->ffn_mult > 0 && (!w->w_up || !w->w_down))))
+    return fail(SANA_ERR_INVALID_ARG, "stack: bf16 weights are NULL");
+  if (mx && (!w->mx_qkvg || !w->mx_qkvg_scales || !w->mx_o || !w->mx_o_scales ||
+             (c->ffn_mult > 0 && (!w->mx_up || !w->mx_up_scales || !w->mx_down ||
+                                  !w->mx_down_scales))))
+    return fail(SANA_ERR_INVALID_ARG, "stack: MX weights are NULL");
   if (c->use_attnres && (!w->w_attn || (c->ffn_mult > 0 && !w->w_ffn)))
     return fail(SANA_ERR_INVALID_ARG, "stack: router queries are NULL");
   if (rope->n_t + rope->n_h + rope->n_w != 64 || rope->H != s->H || rope->W != s->W ||
@@ -148,9 +161,20 @@ extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_sta
   const RopeDev rd{rope->cos_t, rope->sin_t, rope->cos_h, rope->sin_h, rope->cos_w, rope->sin_w,
                    rope->n_t, rope->n_h, rope->n_w};
   const float scale = c->anchor_scale > 0.f ? c->anchor_scale : 1.f / sqrtf(128.f);
+  // one projection x (M, K) . W^T into `outs`: a bf16 GEMM, or the MX
+  // projection (x quantised to MXFP8 into the workspace, MXFP4 weights)
+  auto project = [&](const void* x, int K, int Nout, const void* wbf, const void* wq,
+                     const void* wsc, void* const* outs, int nparts, int epi) -> sana_status {
+    if (!mx) return gemm_run_parts(M, Nout, K, x, K, wbf, outs, nparts, Nout / nparts, epi, st);
+    if (sana_status e = mx_quantize_run(x, M, K, false, P.mxq, P.mxs, st)) return e;
+    return mx_gemm_run_parts(M, Nout, K, P.mxq, P.mxs, wq, wsc, outs, nparts, Nout / nparts, epi,
+                             st);
+  };
+  auto wsel = [&](const void* const* arr, int l) -> const void* { return arr ? arr[l] : nullptr; };
   auto attention = [&](int l) -> sana_status {
     void* parts[4] = {P.q, P.k, P.v, P.g};
-    if (sana_status e = gemm_run_parts(M, 4 * C, C, P.xhat, C, w->w_qkvg[l], parts, 4, C, 0, st))
+    if (sana_status e = project(P.xhat, C, 4 * C, wsel(w->w_qkvg, l), wsel(w->mx_qkvg, l),
+                                wsel(w->mx_qkvg_scales, l), parts, 4, 0))
       return e;
     if (l % c->ratio == c->ratio - 1) {
       if (c->anchor_keep_tiles > 0)
@@ -167,14 +191,22 @@ extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_sta
     // plain pre-norm residual stream in `out`
     if (cudaMemcpyAsync(out, x_embed, (size_t)M * C * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
       return fail(SANA_ERR_CUDA, "stack: copy of the embedding failed");
+    void* o_out[1] = {out};
+    void* f_out[1] = {P.ffn};
     for (int l = 0; l < c->layers; ++l) {
       if (sana_status e = rmsnorm_run(M, C, SANA_BF16, out, c->rms_eps, P.xhat, st)) return e;
       if (sana_status e = attention(l)) return e;
-      if (sana_status e = gemm_run(M, C, C, P.attn, C, w->w_o[l], out, C, 2, st)) return e;
+      if (sana_status e = project(P.attn, C, C, wsel(w->w_o, l), wsel(w->mx_o, l),
+                                  wsel(w->mx_o_scales, l), o_out, 1, 2))
+        return e;
       if (c->ffn_mult > 0) {
         if (sana_status e = rmsnorm_run(M, C, SANA_BF16, out, c->rms_eps, P.xhat, st)) return e;
-        if (sana_status e = gemm_run(M, F, C, P.xhat, C, w->w_up[l], P.ffn, F, 1, st)) return e;
-        if (sana_status e = gemm_run(M, C, F, P.ffn, F, w->w_down[l], out, C, 2, st)) return e;
+        if (sana_status e = project(P.xhat, C, F, wsel(w->w_up, l), wsel(w->mx_up, l),
+                                    wsel(w->mx_up_scales, l), f_out, 1, 1))
+          return e;
+        if (sana_status e = project(P.ffn, F, C, wsel(w->w_down, l), wsel(w->mx_down, l),
+                                    wsel(w->mx_down_scales, l), o_out, 1, 2))
+          return e;
       }
     }
     return SANA_OK;
@@ -197,7 +229,10 @@ extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_sta
                                     w->w_attn, c->rms_eps, nullptr, nullptr, true, P.xhat, st))
       return e;
     if (sana_status e = attention(l)) return e;
-    if (sana_status e = gemm_run(M, C, C, P.attn, C, w->w_o[l], partial, C, partial_live ? 2 : 0, st))
+    void* p_out[1] = {partial};
+    void* f_out[1] = {P.ffn};
+    if (sana_status e = project(P.attn, C, C, wsel(w->w_o, l), wsel(w->mx_o, l),
+                                wsel(w->mx_o_scales, l), p_out, 1, partial_live ? 2 : 0))
       return e;
     partial_live = true;
     if (c->ffn_mult > 0) {
@@ -205,8 +240,12 @@ extern "C" sana_status sana_hybrid_stack_fwd(const sana_shape* s, const sana_sta
       if (sana_status e = attnres_run(s->B, Nseq, C, SANA_BF16, src.data(), (int)src.size(),
                                       w->w_ffn, c->rms_eps, nullptr, nullptr, true, P.xhat, st))
         return e;
-      if (sana_status e = gemm_run(M, F, C, P.xhat, C, w->w_up[l], P.ffn, F, 1, st)) return e;
-      if (sana_status e = gemm_run(M, C, F, P.ffn, F, w->w_down[l], partial, C, 2, st)) return e;
+      if (sana_status e = project(P.xhat, C, F, wsel(w->w_up, l), wsel(w->mx_up, l),
+                                  wsel(w->mx_up_scales, l), f_out, 1, 1))
+        return e;
+      if (sana_status e = project(P.ffn, F, C, wsel(w->w_down, l), wsel(w->mx_down, l),
+                                  wsel(w->mx_down_scales, l), p_out, 1, 2))
+        return e;
     }
     if ((l + 1) % c->block_span == 0) {  // freeze the block summary
       ++nsum;

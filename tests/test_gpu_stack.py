@@ -187,3 +187,81 @@ def test_stack_full_width_and_depth_short_sequence():
     print(f"16-layer stack, N=512, C=3072: max_rel {err:.3e} "
           f"elementwise {orc.elementwise_rel_err(f64(y), yo):.3e}")
     assert err <= BF16_TOL, err
+
+
+def _mx_stack(x, ws, w_attn, w_ffn, grid, heads, cfg, wsd=None, ws_buf=None):
+    rope = sana.Rope(grid[0], grid[1], grid[2], (22, 21, 21))
+    if wsd is None:
+        wsd = sana.mx_quantize_stack_weights([{k: v.cuda() for k, v in d.items()} for d in ws])
+        for d in wsd:  # the MX form alone must suffice
+            for key in ("qkvg", "o", "up", "down"):
+                d.pop(key, None)
+    y = sana.hybrid_stack_fwd(x.cuda(), wsd, w_attn.cuda(), w_ffn.cuda(), rope, grid, heads, cfg,
+                              ws=ws_buf)
+    sana.sync_status()
+    return y, wsd
+
+
+def test_stack_mx_projections_end_to_end():
+    """Four layers without AttnRes or FFN, every projection as the MX projection
+    (MXFP4 weights quantised by the library, activations quantised to MXFP8 on
+    the fly), against the oracle stack with its MX option; C = 256 on a
+    512-token grid.  (Deeper MX stacks are checked teacher-forced below: the
+    quantiser is discontinuous, so a one-ulp bf16 difference upstream moves
+    an element by a whole E4M3 step and the two sides drift apart with depth.)"""
+    grid, heads, C, N, layers = (4, 8, 16), 2, 256, 512, 4
+    x, ws, w_attn, w_ffn = _stack_inputs(C, N, layers, 0, 13204)
+    cfg = sana.stack_config(layers, use_attnres=False, ffn_mult=0, mx_projections=True)
+    y, _ = _mx_stack(x, ws, w_attn, w_ffn, grid, heads, cfg)
+    wo = [{k: f64(v) for k, v in d.items()} for d in ws]
+    yo = orc.hybrid_stack(f64(x), wo, f64(w_attn), f64(w_ffn), grid, (22, 21, 21), heads, layers,
+                          use_attnres=False, ffn=False, mx=True)
+    err = orc.max_rel_err(f64(y), yo)
+    assert err <= BF16_TOL, err
+
+
+def _bf16(a):
+    return f64(torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16))
+
+
+def test_stack_mx_projections_teacher_forced():
+    """Eight layers with AttnRes (blocks of 4) and FFN 3C, MX projections,
+    checked step by step on the GPU's own inputs of each step: the QKVG
+    projection of the routed, normalised input (rounded to bf16 as the GPU
+    stores it before quantising), W_o and the FFN projections of the GPU's
+    attention output and FFN hidden state, and the partial sum."""
+    grid, heads, C, N, layers, span = (4, 8, 16), 2, 256, 512, 8, 4
+    x, ws, w_attn, w_ffn = _stack_inputs(C, N, layers, 3, 13208)
+    wo = [{k: f64(v) for k, v in d.items()} for d in ws]
+    cfg_for = lambda L: sana.stack_config(L, block_span=span, use_attnres=True, ffn_mult=3,
+                                          mx_projections=True)
+    buf = torch.empty(sana.hybrid_stack_workspace_size(1, grid, heads, cfg_for(layers)),
+                      dtype=torch.uint8, device="cuda")
+    wsd = None
+    emb, summaries, partial = f64(x), [], None
+    mx = orc.mx_linear
+    for l in range(layers):
+        cfg = cfg_for(l + 1)
+        _, wsd = _mx_stack(x, ws, w_attn, w_ffn, grid, heads, cfg, wsd, buf)
+        vw = sana.hybrid_stack_workspace_views(buf, 1, grid, heads, cfg)
+        srcs = [emb] + summaries + ([partial] if partial is not None else [])
+        h, _ = orc.attnres_route(srcs, f64(w_attn))
+        xh = _bf16(orc.rmsnorm(h)[0])
+        qkvg = mx(xh, wo[l]["qkvg"])
+        for i, key in enumerate("qkvg"):
+            err = orc.max_rel_err(f64(vw[key])[0], qkvg[:, i * C:(i + 1) * C])
+            assert err <= BF16_TOL, (l, key, err)
+        attn = f64(vw["attn"])[0]
+        mid = _bf16(mx(attn, wo[l]["o"]) + (partial[0] if partial is not None else 0.0))
+        hf, _ = orc.attnres_route([emb] + summaries + [mid[None]], f64(w_ffn))
+        xf = f64(vw["x_hat"])[0]
+        assert orc.max_rel_err(xf, orc.rmsnorm(hf)[0]) <= BF16_TOL, l
+        u = f64(vw["ffn"])[0]
+        assert orc.max_rel_err(u, orc.silu(mx(xf, wo[l]["up"]))) <= BF16_TOL, l
+        nsum = len(summaries)
+        new = f64(vw["blocks"][nsum])
+        assert orc.max_rel_err(new[0], mid + mx(u, wo[l]["down"])) <= BF16_TOL, l
+        partial = new
+        if (l + 1) % span == 0:
+            summaries.append(partial)
+            partial = None

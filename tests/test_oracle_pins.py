@@ -778,3 +778,30 @@ def test_error_measures_hand_worked():
     got2 = np.array([10.0, 1.0, -0.001, 0.003])   # 0.003 / 0.01
     assert orc.elementwise_rel_err(got2, ref) == pytest.approx(0.3, rel=1e-12)
     assert orc.max_rel_err(got2, ref) == pytest.approx(0.0003, rel=1e-12)
+
+
+def test_mx_stack_projections_are_the_mx_linear():
+    """The stack's MX option changes only the projections: with weights whose
+    MX rounding is exact (E2M1 values times a power of two per block), one
+    layer without AttnRes and without FFN
+    equals the exact layer with the activations' MXFP8 rounding applied to
+    the normalised input and to the attention output (quantising along the
+    wrong axis, with the wrong format, or skipping a projection fails)."""
+    grid, split, heads, D = (2, 2, 2), (2, 3, 3), 2, 16
+    C, N = heads * D, 8
+    x = rand(1, N, C)
+    vals = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    pick = lambda *sh: rng.choice(vals, size=sh) * rng.choice([-1.0, 1.0], size=sh) * 2.0 ** -3
+    ws = [dict(qkvg=pick(4 * C, C), o=pick(C, C))]
+    out = orc.hybrid_stack(x, ws, None, None, grid, split, heads, 1, use_attnres=False,
+                           ffn=False, mx=True)
+    q8 = lambda a: orc.mx_dequantize(*orc.mx_quantize(a, orc.E4M3))
+    # the weights are MXFP4-exact: their quantisation is the identity
+    wq = orc.mx_dequantize(*orc.mx_quantize(ws[0]["qkvg"], orc.E2M1))
+    np.testing.assert_array_equal(wq, ws[0]["qkvg"])
+    xh = q8(orc.rmsnorm(x)[0])
+    qkvg = xh @ ws[0]["qkvg"].T
+    q, k, v, g = (qkvg[None, :, i * C:(i + 1) * C] for i in range(4))
+    a = orc.linattn_bruteforce(q, k, v, grid, split, heads, gate=g)
+    ref = x + q8(a[0]) @ ws[0]["o"].T
+    assert rel(out, ref) < 1e-12
