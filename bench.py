@@ -755,6 +755,21 @@ def run_bwd_only(args):
     nb = 9 * TENSOR_BYTES  # q, k, v, g, dy read once; dq, dk, dv, dg written once
     print(json.dumps({"linattn_bwd_720p_ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
                       "GB_per_s": nb / (ms / 1e3) / 1e9}), flush=True)
+    del q, k, v, g, dy
+    # the AttnRes router's backward over 3 sources: 3 sources and dh read,
+    # 3 source gradients written
+    srcs = [t.cuda() for t in si.attnres_sources(5, 3, 1, WL.N, WL.C)]
+    w_attn, _ = (t.cuda() for t in si.router_queries(5, WL.C))
+    dh = si.normal(7100, (1, WL.N, WL.C)).cuda()
+    wsb = torch.empty(sana._lib.lib.sana_attnres_route_bwd_workspace_size(1, WL.N, WL.C),
+                      dtype=torch.uint8, device="cuda")
+    f = lambda: sana.attnres_route_bwd(srcs, w_attn, dh, ws=wsb)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    print(json.dumps({"attnres_route_bwd_720p_3src_ms": ms,
+                      "GB_per_s": 7 * TENSOR_BYTES / (ms / 1e3) / 1e9}), flush=True)
 
 
 def run_sparse_only(args):

@@ -73,6 +73,31 @@ def test_bf16_rescaling_path():
     assert orc.max_rel_err(f64(y), yo) <= BF16_TOL
 
 
+@pytest.mark.parametrize("use_rope", [False, True])
+def test_bf16_large_max_jumps(use_rope):
+    """Row maxima that jump late and far: key tile 0 is zero (logits 0);
+    one key of tile 2 is 3 x a query row (a jump of about 50 in base-2 units
+    for that row, and spread jumps for the others) and one key of tile 4 is
+    10 x another query row (a jump of about 160 for that row, past the range
+    in which 2^(s - m) against a stale reference stays finite).  Every row's
+    softmax must still be exact up to bf16 rounding."""
+    grid, heads = (3, 16, 16), 2
+    N, C = 768, 256
+    q = si.normal(11900, (1, N, C))
+    k, v, g = (si.normal(11901 + i, (1, N, C)) for i in range(3))
+    k[:, :128] = 0
+    k[0, 300] = q[0, 5] * 3
+    k[0, 560] = q[0, 77] * 10
+    split = (22, 21, 21)
+    y = gpu_anchor(q, k, v, g, grid, split, heads, use_rope=use_rope)
+    yo = orc.softmax_anchor(f64(q), f64(k), f64(v), grid if use_rope else None,
+                            split if use_rope else None, heads, gate=f64(g), use_rope=use_rope)
+    err = orc.max_rel_err(f64(y), yo)
+    print(f"anchor large jumps (rope={use_rope}): max_rel {err:.3e}")
+    assert np.isfinite(f64(y)).all()
+    assert err <= BF16_TOL, err
+
+
 @pytest.mark.parametrize("c", [-12.0, -6.0])
 def test_gate_relative_accuracy_at_saturated_logits(c):
     """Every gate logit equal to c: the output is sigmoid(c) times the
