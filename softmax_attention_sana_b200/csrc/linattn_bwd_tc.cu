@@ -87,6 +87,64 @@ __device__ __forceinline__ float2 pair_cs(const GlobalRowRope& rr, int j) {
   return rr.cs(j);
 }
 
+// ---- packed fp32 (f32x2): one instruction for two values
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t bf2_to_pk2(uint32_t u) {
+  return pk2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t pk2_to_bf2(uint64_t v) {
+  float a, b;
+  up2(v, a, b);
+  return f2_to_bf2(a, b);
+}
+// max(x, 0) of both bf16 halves
+__device__ __forceinline__ uint32_t relu_bf2(uint32_t w) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0u));
+  return r;
+}
+// sigmoid of two values, the steps of sigmoid_fast on f32x2 (the same
+// exponential and the same two Newton steps for 1 / (1 + t))
+__device__ __forceinline__ uint64_t sigmoid_pk2(float x0, float x1) {
+  float t0, t1;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t0) : "f"(-1.4426950408889634f * fabsf(x0)));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t1) : "f"(-1.4426950408889634f * fabsf(x1)));
+  const uint64_t t = pk2(t0, t1);
+  const uint64_t d = add2(t, pk2(1.f, 1.f));
+  const uint64_t nd = mul2(d, pk2(-1.f, -1.f));
+  uint64_t r = fma2(pk2(-0.47058823529411764f, -0.47058823529411764f), d,
+                    pk2(1.4117647058823530f, 1.4117647058823530f));
+  r = mul2(r, fma2(nd, r, pk2(2.f, 2.f)));
+  r = mul2(r, fma2(nd, r, pk2(2.f, 2.f)));
+  const uint64_t tr = mul2(t, r);
+  float r0, r1, q0, q1;
+  up2(r, r0, r1);
+  up2(tr, q0, q1);
+  return pk2(x0 >= 0.f ? r0 : q0, x1 >= 0.f ? r1 : q1);
+}
+
 // Rotation by the opposite angle (the transpose of the RoPE rotation).
 __device__ __forceinline__ float2 rotate_t(float x, float y, float2 cs) {
   return make_float2(x * cs.x + y * cs.y, y * cs.x - x * cs.y);
@@ -121,31 +179,36 @@ template <int NT, int NH, int C4, class RR>
 __device__ __forceinline__ float quarter_forward(uint8_t* tile, int r, const RR& rr,
                                                  const float* z, uint32_t& mask) {
   uint8_t* half = tile + (C4 >> 1) * kHalf;
-  float den = 0.f;
+  uint64_t den2 = pk2(0.f, 0.f);  // even and odd columns, summed at the end
   mask = 0;
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     uint4* p = reinterpret_cast<uint4*>(half + sw128_off(r, (C4 & 1) * 4 + ch));
     const uint4 raw = *p;
     uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    float zc[8];
+    if (z) {
+      const float4 z0 = *reinterpret_cast<const float4*>(z + C4 * 32 + ch * 8);
+      const float4 z1 = *reinterpret_cast<const float4*>(z + C4 * 32 + ch * 8 + 4);
+      zc[0] = z0.x; zc[1] = z0.y; zc[2] = z0.z; zc[3] = z0.w;
+      zc[4] = z1.x; zc[5] = z1.y; zc[6] = z1.z; zc[7] = z1.w;
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float2 x = bf2_to_f2(w[i]);
+      const uint32_t xr = relu_bf2(w[i]);  // exact: ReLU commutes with widening
+      const float2 x = bf2_to_f2(xr);
       mask |= (x.x > 0.f ? 1u : 0u) << (ch * 8 + 2 * i);
       mask |= (x.y > 0.f ? 1u : 0u) << (ch * 8 + 2 * i + 1);
-      x.x = fmaxf(x.x, 0.f);
-      x.y = fmaxf(x.y, 0.f);
       const int col = C4 * 32 + ch * 8 + 2 * i;
-      if (z) {
-        den = fmaf(x.x, z[col], den);
-        den = fmaf(x.y, z[col + 1], den);
-      }
+      if (z) den2 = fma2(pk2(x.x, x.y), pk2(zc[2 * i], zc[2 * i + 1]), den2);
       const float2 rt = rotate(x.x, x.y, pair_cs<NT, NH>(rr, col >> 1));
       w[i] = f2_to_bf2(rt.x, rt.y);
     }
     *p = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  return den;
+  float d0, d1;
+  up2(den2, d0, d1);
+  return d0 + d1;
 }
 
 template <int NT, int NH, class RR>
@@ -184,6 +247,11 @@ __device__ __forceinline__ void quarter_backward(uint8_t* tile, int r, const RR&
       uint4* p = reinterpret_cast<uint4*>(half + sw128_off(r, (C4 & 1) * 4 + part * 2 + cc));
       const uint4 raw = *p;
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      const int cb = C4 * 32 + part * 16 + cc * 8;  // first of these 8 columns
+      const float4 z0 = *reinterpret_cast<const float4*>(zz + cb);
+      const float4 z1 = *reinterpret_cast<const float4*>(zz + cb + 4);
+      const float zc[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+      const uint64_t add2v = pk2(add, add);
       uint32_t out[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -193,13 +261,17 @@ __device__ __forceinline__ void quarter_backward(uint8_t* tile, int r, const RR&
         if (zacc) {
           const float2 xr = bf2_to_f2(w[i]);
           const float2 ph = rotate_t(xr.x, xr.y, cs);
-          zacc[j] = fmaf(add, ph.x, zacc[j]);
-          zacc[j + 1] = fmaf(add, ph.y, zacc[j + 1]);
+          float a0, a1;
+          up2(fma2(add2v, pk2(ph.x, ph.y), pk2(zacc[j], zacc[j + 1])), a0, a1);
+          zacc[j] = a0;
+          zacc[j + 1] = a1;
         }
         const float2 gr =
             rotate_t(__uint_as_float(gv[cc * 8 + 2 * i]), __uint_as_float(gv[cc * 8 + 2 * i + 1]), cs);
-        const float g0 = ((mask >> j) & 1u) ? fmaf(add, zz[col], gr.x) : 0.f;
-        const float g1 = ((mask >> (j + 1)) & 1u) ? fmaf(add, zz[col + 1], gr.y) : 0.f;
+        float g0, g1;
+        up2(fma2(add2v, pk2(zc[2 * i], zc[2 * i + 1]), pk2(gr.x, gr.y)), g0, g1);
+        g0 = ((mask >> j) & 1u) ? g0 : 0.f;
+        g1 = ((mask >> (j + 1)) & 1u) ? g1 : 0.f;
         out[i] = f2_to_bf2(g0, g1);
       }
       *p = make_uint4(out[0], out[1], out[2], out[3]);
@@ -456,7 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           1.f / (ctl.den[s][0][r] + ctl.den[s][1][r] + ctl.den[s][2][r] + ctl.den[s][3][r] + eps);
       uint8_t* dhalf = d_st + s * kTileB + hf * kHalf;
       uint8_t* ghalf = g_st + hf * kHalf;
-      float ddot = 0.f;
+      const uint64_t inv2 = pk2(inv, inv);
+      uint64_t ddot2 = pk2(0.f, 0.f);
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         uint32_t nv[16];
@@ -477,25 +550,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t od[4], og[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float2 dyv = bf2_to_f2(dw[i]);
-            const float o0 = __uint_as_float(nv[cc * 8 + 2 * i]) * inv;
-            const float o1 = __uint_as_float(nv[cc * 8 + 2 * i + 1]) * inv;
-            float do0 = dyv.x, do1 = dyv.y;
+            const uint64_t o2 =
+                mul2(pk2(__uint_as_float(nv[cc * 8 + 2 * i]), __uint_as_float(nv[cc * 8 + 2 * i + 1])),
+                     inv2);
+            uint64_t do2 = bf2_to_pk2(dw[i]);
             if (kGate) {
               const float2 gv = bf2_to_f2(gw[i]);
-              const float s0 = sigmoid_fast(gv.x), s1 = sigmoid_fast(gv.y);
-              og[i] = f2_to_bf2(do0 * o0 * s0 * (1.f - s0), do1 * o1 * s1 * (1.f - s1));
-              do0 *= s0;
-              do1 *= s1;
+              const uint64_t s2 = sigmoid_pk2(gv.x, gv.y);
+              const uint64_t oms = fma2(s2, pk2(-1.f, -1.f), pk2(1.f, 1.f));  // 1 - sigma
+              og[i] = pk2_to_bf2(mul2(mul2(do2, o2), mul2(s2, oms)));
+              do2 = mul2(do2, s2);
             }
-            ddot = fmaf(do0, o0, fmaf(do1, o1, ddot));
-            od[i] = f2_to_bf2(do0 * inv, do1 * inv);
+            ddot2 = fma2(do2, o2, ddot2);
+            od[i] = pk2_to_bf2(mul2(do2, inv2));
           }
           *pd = make_uint4(od[0], od[1], od[2], od[3]);
           if (kGate) *pg = make_uint4(og[0], og[1], og[2], og[3]);
         }
       }
-      ctl.dden[it & 1][c4][r] = -ddot * inv;
+      float dd0, dd1;
+      up2(ddot2, dd0, dd1);
+      ctl.dden[it & 1][c4][r] = -(dd0 + dd1) * inv;
       fence_proxy_async_smem();
       mbar_arrive(&ctl.dnum_ready);
     };
