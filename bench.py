@@ -351,7 +351,15 @@ def components(sana, args):
     ms = time_loop(f, 20)
     out["linattn_bwd_720p"] = {"ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
                                "GB_per_s": 9 * TENSOR_BYTES / (ms / 1e3) / 1e9}
-    del q, k, v, g, dy
+    # the same backward given the forward's state (k, v not read a second time)
+    S, z = sana.linattn_state(k, v, rope, (WL.T, WL.H, WL.W), WL.heads)
+    f = lambda: sana.linattn_bwd(q, k, v, g, rope, (WL.T, WL.H, WL.W), WL.heads, dy, S=S, z=z)
+    for _ in range(3):
+        f()
+    ms = time_loop(f, 20)
+    out["linattn_bwd_saved_state_720p"] = {"ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
+                                           "GB_per_s": 9 * TENSOR_BYTES / (ms / 1e3) / 1e9}
+    del q, k, v, g, dy, S, z
     # projection GEMM of the stack: QKVG at 720p, (75,600 x 3072) . (12,288 x 3072)^T
     A = torch.randn(WL.N, WL.C, device="cuda", dtype=torch.bfloat16)
     Wq = torch.randn(4 * WL.C, WL.C, device="cuda", dtype=torch.bfloat16) * WL.C ** -0.5
@@ -755,7 +763,15 @@ def run_bwd_only(args):
     nb = 9 * TENSOR_BYTES  # q, k, v, g, dy read once; dq, dk, dv, dg written once
     print(json.dumps({"linattn_bwd_720p_ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
                       "GB_per_s": nb / (ms / 1e3) / 1e9}), flush=True)
-    del q, k, v, g, dy
+    S, z = sana.linattn_state(k, v, rope, grid, WL.heads)
+    f = lambda: sana.linattn_bwd(q, k, v, g, rope, grid, WL.heads, dy, S=S, z=z)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    print(json.dumps({"linattn_bwd_saved_state_720p_ms": ms, "tokens_per_s": WL.N / (ms / 1e3),
+                      "GB_per_s": nb / (ms / 1e3) / 1e9}), flush=True)
+    del q, k, v, g, dy, S, z
     # the AttnRes router's backward over 3 sources: 3 sources and dh read,
     # 3 source gradients written
     srcs = [t.cuda() for t in si.attnres_sources(5, 3, 1, WL.N, WL.C)]

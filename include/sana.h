@@ -156,6 +156,20 @@ SANA_API sana_status sana_linattn_bwd(const sana_shape* shape, sana_dtype dtype,
                                       const sana_rope* rope, float eps, const void* dy, void* dq,
                                       void* dk, void* dv, void* d_gate, void* ws, size_t ws_bytes,
                                       sana_stream_t stream);
+/* The same backward for a state the forward already holds: S (device fp32
+ * [B][heads][D][D], S[d][e]) and z (device fp32 [B][heads][D]) exactly as
+ * sana_linattn_state wrote them for these k, v (the two-phase forward keeps
+ * them), so k and v are not read a second time to rebuild them.  Read only;
+ * 16-byte aligned; they must not alias a gradient.  Arguments, workspace,
+ * errors and determinism as for sana_linattn_bwd; NULL S or z is
+ * SANA_ERR_INVALID_ARG. */
+SANA_API sana_status sana_linattn_bwd_saved_state(const sana_shape* shape, sana_dtype dtype,
+                                                  const void* q, const void* k, const void* v,
+                                                  const void* gate_logits, const sana_rope* rope,
+                                                  float eps, const float* S, const float* z,
+                                                  const void* dy, void* dq, void* dk, void* dv,
+                                                  void* d_gate, void* ws, size_t ws_bytes,
+                                                  sana_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * One block of block-causal linear attention with the constant-memory state

@@ -100,6 +100,11 @@ def _load():
         "sana_linattn_bwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                      POINTER(RopeStruct), c_float, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+        "sana_linattn_bwd_saved_state": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p,
+                                                 c_void_p, c_void_p, POINTER(RopeStruct), c_float,
+                                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                 c_void_p, c_void_p, c_void_p, c_size_t,
+                                                 c_void_p]),
         "sana_softmax_anchor_workspace_size": (c_size_t, [POINTER(Shape), c_int]),
         "sana_softmax_anchor_fwd": (c_int, [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, POINTER(RopeStruct), c_float, c_void_p,
@@ -299,11 +304,14 @@ def linattn_block_causal_step(q, k, v, gate, rope: Rope, grid, t_offset, heads, 
     return out
 
 
-def linattn_bwd(q, k, v, gate, rope: Rope, grid, heads, dy, eps=1e-6, ws=None):
+def linattn_bwd(q, k, v, gate, rope: Rope, grid, heads, dy, eps=1e-6, ws=None, S=None, z=None):
     """Gradients (dq, dk, dv, dgate) of the gated linear-attention layer for dY
-    (dgate is None for the ungated layer).  bf16."""
+    (dgate is None for the ungated layer).  bf16.  S, z: the forward's state
+    as linattn_state returned it for these k, v (then it is not rebuilt)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (dy, "dy")):
         _need(t, n)
+    if (S is None) != (z is None):
+        raise ValueError("linattn_bwd: give both S and z or neither")
     B, N, C = q.shape
     D = C // heads
     dt = _dtype_code(q)
@@ -312,9 +320,15 @@ def linattn_bwd(q, k, v, gate, rope: Rope, grid, heads, dy, eps=1e-6, ws=None):
     dg = None if gate is None else torch.empty_like(gate)
     if ws is None:
         ws = _ws(lib.sana_linattn_bwd_workspace_size(ctypes.byref(s), dt), q.device)
-    check(lib.sana_linattn_bwd(
-        ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(rope.struct), eps,
-        _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(), _stream()))
+    if S is None:
+        check(lib.sana_linattn_bwd(
+            ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(rope.struct),
+            eps, _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws), ws.numel(), _stream()))
+    else:
+        check(lib.sana_linattn_bwd_saved_state(
+            ctypes.byref(s), dt, _ptr(q), _ptr(k), _ptr(v), _ptr(gate), ctypes.byref(rope.struct),
+            eps, _ptr(S), _ptr(z), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(ws),
+            ws.numel(), _stream()))
     return dq, dk, dv, dg
 
 

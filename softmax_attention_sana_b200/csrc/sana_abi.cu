@@ -348,10 +348,11 @@ size_t linattn_bwd_ws_bytes(const sana_shape& s) {
   return 2 * one;
 }
 
+// S_saved / z_saved: the forward's combined state, or NULL to rebuild it from k, v.
 sana_status linattn_bwd_run(const sana_shape& s, const void* q, const void* k, const void* v,
                             const void* gt, const void* dy, const RopeDev& rope, float eps,
-                            void* dq, void* dk, void* dv, void* dg, void* ws, size_t ws_bytes,
-                            cudaStream_t st) {
+                            const float* S_saved, const float* z_saved, void* dq, void* dk,
+                            void* dv, void* dg, void* ws, size_t ws_bytes, cudaStream_t st) {
   const GridDev g = to_grid(s);
   if (g.N == 0) return SANA_OK;
   const size_t one = carve_linattn(s, SANA_BF16, nullptr).bytes;
@@ -363,11 +364,17 @@ sana_status linattn_bwd_run(const sana_shape& s, const void* q, const void* k, c
   const LinWs fw = carve_linattn(s, SANA_BF16, ws);
   const LinWs bw = carve_linattn(s, SANA_BF16, static_cast<char*>(ws) + one);
   const LinAttnPlan plan = linattn_plan(s, SANA_BF16);
-  if (sana_status e = linattn_bf16_state(s, plan, k, v, rope, g, nullptr, nullptr, nullptr, nullptr,
-                                         fw.ws_S, fw.ws_z, fw.S_f32, fw.z_comb, st))
-    return e;
-  return linattn_bf16_backward(s, plan, q, k, v, gt, dy, rope, g, eps, fw.S_f32, fw.z_comb,
-                               bw.ws_S, bw.ws_z, bw.S_f32, bw.z_comb, dq, dk, dv, dg, st);
+  const float* S = S_saved;
+  const float* z = z_saved;
+  if (!S) {
+    if (sana_status e = linattn_bf16_state(s, plan, k, v, rope, g, nullptr, nullptr, nullptr,
+                                           nullptr, fw.ws_S, fw.ws_z, fw.S_f32, fw.z_comb, st))
+      return e;
+    S = fw.S_f32;
+    z = fw.z_comb;
+  }
+  return linattn_bf16_backward(s, plan, q, k, v, gt, dy, rope, g, eps, S, z, bw.ws_S, bw.ws_z,
+                               bw.S_f32, bw.z_comb, dq, dk, dv, dg, st);
 }
 
 // ---------------------------------------------------------------- anchor
@@ -572,11 +579,12 @@ size_t sana_linattn_bwd_workspace_size(const sana_shape* s, sana_dtype dt) {
   return linattn_bwd_ws_bytes(*s);
 }
 
-sana_status sana_linattn_bwd(const sana_shape* s, sana_dtype dt, const void* q, const void* k,
-                             const void* v, const void* g, const sana_rope* rope, float eps,
-                             const void* dy, void* dq, void* dk, void* dv, void* dg, void* ws,
-                             size_t ws_bytes, sana_stream_t stream) {
-  const char* who = "sana_linattn_bwd";
+// Validation shared by both backward entry points (S, z NULL for the first).
+static sana_status bwd_checked_run(const char* who, bool saved, const sana_shape* s, sana_dtype dt,
+                            const void* q, const void* k, const void* v, const void* g,
+                            const sana_rope* rope, float eps, const float* S, const float* z,
+                            const void* dy, void* dq, void* dk, void* dv, void* dg, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
   if (sana_status e = check_shape(s, dt, who)) return e;
   if (dt != SANA_BF16) return fail(SANA_ERR_UNSUPPORTED, "%s: bf16 only", who);
   if (sana_status e = check_rope(rope, s, who)) return e;
@@ -599,13 +607,46 @@ sana_status sana_linattn_bwd(const sana_shape* s, sana_dtype dt, const void* q, 
     for (const void* o2 : outs)
       if (o2 != o && overlap(o, n, o2, n)) return fail(SANA_ERR_INVALID_ARG, "%s: gradients alias each other", who);
   }
+  if (saved) {
+    if (!S || !z) return fail(SANA_ERR_INVALID_ARG, "%s: saved state S, z must be given", who);
+    if (!aligned16(S) || !aligned16(z))
+      return fail(SANA_ERR_INVALID_ARG, "%s: state must be 16-byte aligned", who);
+    const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
+    const size_t zb = (size_t)s->B * s->heads * s->head_dim * 4;
+    for (const void* o : outs)
+      if (o && (overlap(o, n, S, sb) || overlap(o, n, z, zb)))
+        return fail(SANA_ERR_INVALID_ARG, "%s: a gradient aliases the saved state", who);
+  }
   const size_t need = linattn_bwd_ws_bytes(*s);
   if (!ws || ws_bytes < need)
     return fail(SANA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws ? ws_bytes : 0, need);
   if (reinterpret_cast<uintptr_t>(ws) & 255u)
     return fail(SANA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
-  return linattn_bwd_run(*s, q, k, v, g, dy, to_dev(*rope), eps, dq, dk, dv, dg, ws, ws_bytes,
-                         stream);
+  if (saved) {
+    const size_t sb = (size_t)s->B * s->heads * s->head_dim * s->head_dim * 4;
+    if (overlap(ws, ws_bytes, S, sb) || overlap(ws, ws_bytes, z, (size_t)s->B * s->heads * s->head_dim * 4))
+      return fail(SANA_ERR_INVALID_ARG, "%s: the workspace overlaps the saved state", who);
+  }
+  return linattn_bwd_run(*s, q, k, v, g, dy, to_dev(*rope), eps, saved ? S : nullptr,
+                         saved ? z : nullptr, dq, dk, dv, dg, ws, ws_bytes, stream);
+}
+
+sana_status sana_linattn_bwd(const sana_shape* s, sana_dtype dt, const void* q, const void* k,
+                             const void* v, const void* g, const sana_rope* rope, float eps,
+                             const void* dy, void* dq, void* dk, void* dv, void* dg, void* ws,
+                             size_t ws_bytes, sana_stream_t stream) {
+  return bwd_checked_run("sana_linattn_bwd", false, s, dt, q, k, v, g, rope, eps, nullptr, nullptr,
+                         dy, dq, dk, dv, dg, ws, ws_bytes, stream);
+}
+
+sana_status sana_linattn_bwd_saved_state(const sana_shape* s, sana_dtype dt, const void* q,
+                                         const void* k, const void* v, const void* g,
+                                         const sana_rope* rope, float eps, const float* S,
+                                         const float* z, const void* dy, void* dq, void* dk,
+                                         void* dv, void* dg, void* ws, size_t ws_bytes,
+                                         sana_stream_t stream) {
+  return bwd_checked_run("sana_linattn_bwd_saved_state", true, s, dt, q, k, v, g, rope, eps, S, z,
+                         dy, dq, dk, dv, dg, ws, ws_bytes, stream);
 }
 
 size_t sana_linattn_block_causal_scan_workspace_size(const sana_shape* s, int chunk_frames,

@@ -142,8 +142,8 @@ sana_status linattn_bf16_backward(const sana_shape& s, const LinAttnPlan& plan, 
 size_t linattn_bwd_ws_bytes(const sana_shape& s);
 sana_status linattn_bwd_run(const sana_shape& s, const void* q, const void* k, const void* v,
                             const void* gt, const void* dy, const RopeDev& rope, float eps,
-                            void* dq, void* dk, void* dv, void* dg, void* ws, size_t ws_bytes,
-                            cudaStream_t st);
+                            const float* S_saved, const float* z_saved, void* dq, void* dk,
+                            void* dv, void* dg, void* ws, size_t ws_bytes, cudaStream_t st);
 
 // Bidirectional (S_prev == nullptr) or block-causal step.
 sana_status linattn_run(const sana_shape& s, sana_dtype dt, const void* q, const void* k,

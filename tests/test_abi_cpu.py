@@ -176,6 +176,17 @@ def test_backward_validation():
     assert call(dq=2 * M) == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
     assert call(ws_bytes=64) == L.SANA_ERR_WORKSPACE
 
+    def saved(S=9 * M, z=10 * M, dq=5 * M, ws=1 << 28):
+        return L.lib.sana_linattn_bwd_saved_state(
+            ctypes.byref(s), L.SANA_BF16, M, 2 * M, 3 * M, None, ctypes.byref(r), 1e-6, S, z,
+            4 * M, dq, 6 * M, 7 * M, None, ws, 1 << 26, None)
+    assert saved(S=None) == L.SANA_ERR_INVALID_ARG and "saved state" in L.last_error()
+    assert saved(z=None) == L.SANA_ERR_INVALID_ARG
+    assert saved(S=9 * M + 4) == L.SANA_ERR_INVALID_ARG and "aligned" in L.last_error()
+    assert saved(dq=9 * M) == L.SANA_ERR_INVALID_ARG and "saved state" in L.last_error()
+    assert saved(ws=9 * M) == L.SANA_ERR_INVALID_ARG and "workspace" in L.last_error()
+    assert saved(dq=2 * M) == L.SANA_ERR_INVALID_ARG and "alias" in L.last_error()
+
 
 def test_attnres_and_gemm_validation():
     L = _lib

@@ -52,6 +52,21 @@ def test_small_ragged_matches_the_oracle(B, grid, heads, split, gated):
         assert e <= BF16_TOL, (name, e)
 
 
+def test_saved_state_equals_recomputed_state():
+    """The backward given the forward's (S, z) (sana_linattn_bwd_saved_state)
+    runs the same kernels on the same state as the one that rebuilds it."""
+    grid, heads = (3, 9, 16), 2
+    N = grid[0] * grid[1] * grid[2]
+    q, k, v, g, dy = (si.normal(9720 + i, (1, N, heads * 128)).cuda() for i in range(5))
+    rope = sana.Rope(*grid, (22, 21, 21))
+    S, z = sana.linattn_state(k, v, rope, grid, heads)
+    a = sana.linattn_bwd(q, k, v, g, rope, grid, heads, dy)
+    b = sana.linattn_bwd(q, k, v, g, rope, grid, heads, dy, S=S, z=z)
+    sana.sync_status()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 def test_deterministic_and_empty_grid():
     H, W, heads = 9, 16, 2
     N = 4 * H * W
