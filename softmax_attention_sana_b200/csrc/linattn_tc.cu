@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                        const __grid_constant__ CUtensorMap tm_g,
                        const __grid_constant__ CUtensorMap tm_y, const float* __restrict__ S_all,
                        const float* __restrict__ z_all, RopeDev rope, GridDev g, int tiles_total,
-                       int splits, float eps, int* status) {
+                       int splits, float eps, int prefetch, int* status) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ OutSmemCtl ctl;
   uint8_t* smem = align1024(smem_raw);
@@ -441,6 +441,25 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     mbar_init(&ctl.wsync, kWorkers);
     ctl.abort_flag = 0;
     mbar_fence_init();
+    if (prefetch) {
+      // Q and G are inputs of the whole call, complete before its first
+      // kernel started: their first tiles load while the previous launch
+      // (which produces S and z) finishes
+      fence_proxy_async_smem();
+      for (int it = 0; it < kStagesQ && it < ntiles; ++it) {
+        const int n0 = (tile0 + it) * kRows;
+        mbar_arrive_expect_tx(&ctl.fullQ[it], kTileB);
+        tma_load_3d(q_st + it * kTileB, &tm_q, &ctl.fullQ[it], h * kD, n0, b);
+        tma_load_3d(q_st + it * kTileB + kHalf, &tm_q, &ctl.fullQ[it], h * kD + 64, n0, b);
+      }
+      if (kGate)
+        for (int it = 0; it < kStagesG && it < ntiles; ++it) {
+          const int n0 = (tile0 + it) * kRows;
+          mbar_arrive_expect_tx(&ctl.fullG[it], kTileB);
+          tma_load_3d(g_st + it * kTileB, &tm_g, &ctl.fullG[it], h * kD, n0, b);
+          tma_load_3d(g_st + it * kTileB + kHalf, &tm_g, &ctl.fullG[it], h * kD + 64, n0, b);
+        }
+    }
   }
   if (warp == kWarpMmaB) {
     tmem_alloc(&ctl.tmem, 256);
@@ -477,7 +496,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     // ---------------- Q producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
-      for (int it = 0; it < ntiles; ++it) {
+      for (int it = prefetch ? kStagesQ : 0; it < ntiles; ++it) {
         const int s = it % kStagesQ;
         if (it >= kStagesQ && !mbar_wait(&ctl.emptyQ[s], ((it / kStagesQ) - 1) & 1, wc, 0x21))
           break;
@@ -512,7 +531,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           if (!okp) break;
           bulk_wait_read0();  // the stage has been read out
         }
-        if (kGate) {
+        if (kGate && prefetch && it < kStagesG) {
+          // loaded before the launch waited
+        } else if (kGate) {
           const int n0 = (tile0 + it) * kRows;
           mbar_arrive_expect_tx(&ctl.fullG[s], kTileB);
           tma_load_3d(g_st + s * kTileB, &tm_g, &ctl.fullG[s], h * kD, n0, b);
@@ -712,7 +733,7 @@ sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, con
 sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, const void* q,
                                const void* gt, const RopeDev& rope, const GridDev& g,
                                const float* S_f32, const float* z, float eps, void* out,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool prefetch_inputs) {
   const uint64_t C = (uint64_t)s.heads * kD, N = (uint64_t)g.N;
   CUtensorMap tq, tg, ty;
   bool okm = make_tmap_bf16_3d(&tq, q, C, N, s.B, C, N * C, kRows) &&
@@ -731,7 +752,8 @@ sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, con
                  : (stdsp ? linattn_out_kernel<false, kStdNT, kStdNH>
                           : linattn_out_kernel<false, -1, -1>);
   const cudaError_t e = launch_dependent(kern, grid, dim3(kThreadsB), smem_b, st, tq, tg, ty, S_f32,
-                                         z, rope, g, plan.tiles, plan.splits_b, eps, sw);
+                                         z, rope, g, plan.tiles, plan.splits_b, eps,
+                                         prefetch_inputs ? 1 : 0, sw);
   if (e != cudaSuccess) return fail(SANA_ERR_CUDA, "linattn_out_kernel: %s", cudaGetErrorString(e));
   return check_launch("linattn_out_kernel");
 }

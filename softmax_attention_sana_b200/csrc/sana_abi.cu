@@ -271,13 +271,14 @@ sana_status state_phase(const sana_shape& s, sana_dtype dt, const void* k, const
 
 sana_status apply_phase(const sana_shape& s, sana_dtype dt, const void* q, const void* gt,
                         const RopeDev& rope, const GridDev& g, const float* S, const float* z,
-                        float eps, void* out, cudaStream_t st) {
+                        float eps, void* out, cudaStream_t st, bool prefetch_inputs) {
   if (dt == SANA_BF16) {
     if (rope_smem_bytes(g, rope) > kRopeSmemMax)
       return fail(SANA_ERR_UNSUPPORTED,
                   "linear attention: grid %dx%dx%d needs %zu B of RoPE tables (max %zu)", g.T, g.H,
                   g.W, rope_smem_bytes(g, rope), kRopeSmemMax);
-    return linattn_bf16_apply(s, linattn_plan(s, dt), q, gt, rope, g, S, z, eps, out, st);
+    return linattn_bf16_apply(s, linattn_plan(s, dt), q, gt, rope, g, S, z, eps, out, st,
+                              prefetch_inputs);
   }
   return linattn_f32_apply(s, static_cast<const float*>(q), static_cast<const float*>(gt), rope,
                            g, S, z, eps, static_cast<float*>(out), st);
@@ -311,7 +312,9 @@ sana_status linattn_run(const sana_shape& s, sana_dtype dt, const void* q, const
   if (sana_status e = state_phase(s, dt, k, v, rope, g, S_prev, z_prev, S_commit, z_commit, w,
                                   w.S_f32, w.z_comb, st))
     return e;
-  return apply_phase(s, dt, q, gt, rope, g, w.S_f32, w.z_comb, eps, out, st);
+  // the state phase's first kernel is an ordinary launch: q and gt are
+  // complete when the output kernel starts
+  return apply_phase(s, dt, q, gt, rope, g, w.S_f32, w.z_comb, eps, out, st, true);
 }
 
 sana_status linattn_state_run(const sana_shape& s, sana_dtype dt, const void* k, const void* v,
@@ -337,7 +340,7 @@ sana_status linattn_apply_run(const sana_shape& s, sana_dtype dt, const void* q,
                               void* out, cudaStream_t st) {
   const GridDev g = to_grid(s);
   if (g.N == 0) return SANA_OK;
-  return apply_phase(s, dt, q, gt, rope, g, S, z, eps, out, st);
+  return apply_phase(s, dt, q, gt, rope, g, S, z, eps, out, st, false);
 }
 
 // ---------------------------------------------------------------- backward (bf16)

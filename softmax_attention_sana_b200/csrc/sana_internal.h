@@ -113,10 +113,13 @@ sana_status linattn_bf16_state(const sana_shape& s, const LinAttnPlan& plan, con
                                const float* S_prev, const float* z_prev, float* S_state,
                                float* z_state, float* ws_S, float* ws_z, float* S_f32,
                                float* z_out, cudaStream_t st);
+// prefetch_inputs: the first Q / G tiles may be loaded before the launch
+// waits for the previous one (only where q and gt are known to be complete
+// when the call's first, ordinarily launched kernel starts).
 sana_status linattn_bf16_apply(const sana_shape& s, const LinAttnPlan& plan, const void* q,
                                const void* gt, const RopeDev& rope, const GridDev& g,
                                const float* S_f32, const float* z, float eps, void* out,
-                               cudaStream_t st);
+                               cudaStream_t st, bool prefetch_inputs = false);
 int linattn_f32_splits(const sana_shape& s, int N);
 sana_status linattn_f32_state(const sana_shape& s, const float* k, const float* v,
                               const RopeDev& rope, const GridDev& g, int splits,
