@@ -197,6 +197,18 @@ __global__ void __launch_bounds__(kThreadsA, 1)
     mbar_init(&ctl.done, 1);
     ctl.abort_flag = 0;
     mbar_fence_init();
+    // K and V are inputs of an ordinarily launched kernel, complete when it
+    // starts: the first stages load while the RoPE tables are staged
+    fence_proxy_async_smem();
+    for (int it = 0; it < kStagesA && it < ntiles; ++it) {
+      const int n0 = (tile0 + it) * kRows;
+      uint8_t* st = stages + it * 2 * kTileB;
+      mbar_arrive_expect_tx(&ctl.full[it], 2 * kTileB);
+      tma_load_3d(st, &tm_k, &ctl.full[it], h * kD, n0, b);
+      tma_load_3d(st + kHalf, &tm_k, &ctl.full[it], h * kD + 64, n0, b);
+      tma_load_3d(st + kTileB, &tm_v, &ctl.full[it], h * kD, n0, b);
+      tma_load_3d(st + kTileB + kHalf, &tm_v, &ctl.full[it], h * kD + 64, n0, b);
+    }
   }
   if (warp == kWarpMmaA) {
     tmem_alloc(&ctl.tmem, 128);
@@ -211,10 +223,8 @@ __global__ void __launch_bounds__(kThreadsA, 1)
   if (warp == kWarpProdA) {
     // ---------------- TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      int issued = 0;
-      for (int it = 0; it < ntiles; ++it) {
+      int issued = ntiles < kStagesA ? ntiles : kStagesA;  // loaded at the start
+      for (int it = kStagesA; it < ntiles; ++it) {
         const int s = it % kStagesA;
         if (it >= kStagesA && !mbar_wait(&ctl.empty[s], ((it / kStagesA) - 1) & 1, wc, 0x11))
           break;
@@ -466,7 +476,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     tmem_relinquish();
   }
   // everything above overlaps the previous launch's tail; S and z (and Q, G)
-  // are read only after it has finished
+  // are read only after it has finished.  Where the call's inputs are known
+  // complete (prefetch), the RoPE tables are staged before the wait too.
+  RopeSmem rs{};
+  if (prefetch) rs = rope_stage(rope_base, rope, g, b, tid, kThreadsB);
   griddep_wait();
   if (tid < kD) ctl.z[tid] = z_all[(size_t)bh * kD + tid];
   if (tid < kWorkers) {
@@ -486,7 +499,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
     fence_proxy_async_smem();
   }
-  const RopeSmem rs = rope_stage(rope_base, rope, g, b, tid, kThreadsB);
+  if (!prefetch) rs = rope_stage(rope_base, rope, g, b, tid, kThreadsB);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
