@@ -65,6 +65,14 @@ def tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def tensor_peak_sustained():
+    """Dense bf16 tensor peak held for seconds under the power cap, or None."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p)).get("bf16_tflops_sustained")
+    return None
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in ("linattn_tc.cu", "sana_common.cuh", "rope_dev.cuh", "pdl.cuh"):
@@ -434,6 +442,10 @@ def components(sana, args):
                        "peak_kind": tp_kind + " burst (cuBLAS bf16)", "spec_peak": SPEC_BF16_TFLOPS,
                        "spec_frac": ach / SPEC_BF16_TFLOPS, "traffic": None,
                        "algorithmic_flops_per_launch": flops, "ms_per_launch": ms_att}
+        sus = tensor_peak_sustained()
+        if sus:  # context: the same GEMM held for seconds under the power cap
+            anchor_roof["sustained_peak"] = sus
+            anchor_roof["sustained_frac"] = ach / sus
         out["_anchor_roofline"] = anchor_roof
         # the whole call (prepass + kernel)
         f = lambda: sana.softmax_anchor_fwd(q, k, v, g, rope, grid, WL.heads, out=y, ws=ws)
