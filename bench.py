@@ -824,6 +824,23 @@ def run_sparse_only(args):
                       "TFLOP_per_s_executed": kept / (ms / 1e3) / 1e12}), flush=True)
 
 
+def run_gemm_only(args):
+    """The bf16 QKVG projection GEMM of the 720p stack ((75,600 x 3072) .
+    (12,288 x 3072)^T): K steps."""
+    import softmax_attention_sana_b200 as sana
+    A = torch.randn(WL.N, WL.C, device="cuda", dtype=torch.bfloat16)
+    W = torch.randn(4 * WL.C, WL.C, device="cuda", dtype=torch.bfloat16) * WL.C ** -0.5
+    Y = torch.empty(WL.N, 4 * WL.C, device="cuda", dtype=torch.bfloat16)
+    f = lambda: sana.gemm_bf16(A, W, out=Y)
+    for _ in range(args.warmup):
+        f()
+    ms = time_loop(f, args.steps)
+    sana.sync_status()
+    flops = 2 * WL.N * 4 * WL.C * WL.C
+    print(json.dumps({"gemm_qkvg_720p_ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}),
+          flush=True)
+
+
 def run_mx_only(args):
     """The MX projection of the 720p QKVG shape (75,600 x 3072 activations
     quantised on the fly against 12,288 x 3072 MXFP4 weights): K steps."""
@@ -868,6 +885,8 @@ def main():
                     help="run only the linear-attention backward at 720p/5s")
     ap.add_argument("--sparse-only", action="store_true",
                     help="run only the block-sparse anchor at 720p/5s (25%% of the key tiles)")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="only the bf16 QKVG projection GEMM at 720p")
     ap.add_argument("--mx-only", action="store_true",
                     help="run only the MX projection of the 720p QKVG shape")
     ap.add_argument("--chunk-only", action="store_true",
@@ -895,6 +914,9 @@ def main():
             return
         if args.mx_only:
             run_mx_only(args)
+            return
+        if args.gemm_only:
+            run_gemm_only(args)
             return
         if args.impl == "reference":
             run_reference(args, world, rank)
