@@ -72,6 +72,33 @@ def test_bf16_small_with_ragged_tails(B, heads, grid):
     assert orc.max_rel_err(f64(y), yo) <= BF16_TOL
 
 
+@pytest.mark.parametrize("gated", [True, False])
+def test_two_phases_equal_the_fused_layer(gated):
+    """sana_linattn_state then sana_linattn_apply (the standalone output pass,
+    which loads nothing before its launch dependency resolves) give the fused
+    layer's output bit for bit, and the state (S, z) matches the oracle's."""
+    B, heads, grid = 2, 2, (3, 9, 16)
+    N = grid[0] * grid[1] * grid[2]
+    q, k, v, g = (si.normal(10900 + i, (B, N, heads * 128)) for i in range(4))
+    if not gated:
+        g = None
+    rope = sana.Rope(*grid, (22, 21, 21))
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    gc = None if g is None else g.cuda()
+    y1 = sana.linattn_fwd(qc, kc, vc, gc, rope, grid, heads)
+    S, z = sana.linattn_state(kc, vc, rope, grid, heads)
+    y2 = sana.linattn_apply(qc, gc, rope, grid, heads, S, z)
+    sana.sync_status()
+    assert torch.equal(y1, y2)
+    ang = orc.rope_angles(*grid, 22, 21, 21)
+    So, zo = orc.linattn_state(f64(k), f64(v), ang, heads)
+    assert orc.max_rel_err(S.cpu().double().numpy(), So) <= BF16_TOL
+    assert orc.max_rel_err(z.cpu().double().numpy(), zo) <= BF16_TOL
+    yo, _, _ = orc.linattn_bidirectional(f64(q), f64(k), f64(v), grid, (22, 21, 21), heads,
+                                         gate=None if g is None else f64(g))
+    assert orc.max_rel_err(f64(y2), yo) <= BF16_TOL
+
+
 def test_empty_grid_is_a_no_op():
     rope = sana.Rope(1, 4, 4, (22, 21, 21))
     q = torch.zeros(1, 0, 256, dtype=torch.bfloat16, device="cuda")
