@@ -717,9 +717,10 @@ def run_chunk_only(args):
 
 
 def run_anchor_only(args):
-    """The softmax anchor on the 480p grid (N = 32,760): K steps, ms per call."""
+    """The softmax anchor on the 480p grid (N = 32,760), or with --anchor-720p
+    on the 720p/5s grid (N = 75,600): K steps, ms per call."""
     import softmax_attention_sana_b200 as sana
-    wl = si.P480
+    wl = si.P720 if args.anchor_720p else si.P480
     q, k, v, g = (t.cuda() for t in si.qkvg(wl))
     rope = sana.Rope(wl.T, wl.H, wl.W, wl.rope_split)
     y = torch.empty_like(q)
@@ -729,7 +730,8 @@ def run_anchor_only(args):
     ms = time_loop(f, args.steps)
     sana.sync_status()
     flops = 4 * wl.N * wl.N * wl.heads * wl.D
-    print(json.dumps({"anchor_480p_ms": ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}), flush=True)
+    name = "anchor_720p_ms" if args.anchor_720p else "anchor_480p_ms"
+    print(json.dumps({name: ms, "TFLOP_per_s": flops / (ms / 1e3) / 1e12}), flush=True)
 
 
 def run_scan_only(args):
@@ -885,6 +887,8 @@ def main():
                     help="run only the linear-attention backward at 720p/5s")
     ap.add_argument("--sparse-only", action="store_true",
                     help="run only the block-sparse anchor at 720p/5s (25%% of the key tiles)")
+    ap.add_argument("--anchor-720p", action="store_true",
+                    help="with --anchor-only: the 720p/5s grid instead of 480p")
     ap.add_argument("--gemm-only", action="store_true",
                     help="only the bf16 QKVG projection GEMM at 720p")
     ap.add_argument("--mx-only", action="store_true",
