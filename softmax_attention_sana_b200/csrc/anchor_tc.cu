@@ -493,17 +493,13 @@ sana_status anchor_bf16_run(const sana_shape& s, const void* qr, const void* kr,
   if (gt) okm = okm && make_tmap_bf16_3d(&tg, gt, C, N, s.B, C, N * C, kRows);
   else tg = tq;
   if (!okm) return fail(SANA_ERR_CUDA, "anchor: cuTensorMapEncodeTiled failed");
-  static bool attr[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr[dev]) {
+  once_per_context(kAttrAnchor, [] {
     const int bytes = (int)kAnchorSmem;
     cudaFuncSetAttribute(anchor_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     cudaFuncSetAttribute(anchor_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     cudaFuncSetAttribute(anchor_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     cudaFuncSetAttribute(anchor_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    attr[dev] = true;
-  }
+  });
   const int qtiles = (g.N + kRows - 1) / kRows;
   const dim3 grid((qtiles + 1) / 2, s.heads, s.B);
   int* sw = status_word();

@@ -231,13 +231,9 @@ sana_status gemm_run_parts(long long M, int N, int K, const void* A, long long l
   for (int i = 0; i < nparts; ++i) o.part[i] = static_cast<__nv_bfloat16*>(outs[i]);
   o.part_cols = N / nparts;
   o.ldo = ldo;
-  static bool attr[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr[dev]) {
+  once_per_context(kAttrGemm, [] {
     cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
-    attr[dev] = true;
-  }
+  });
   const long long tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int pairs = (int)(tiles < kNumSMs / 2 ? tiles : kNumSMs / 2);
   gemm_kernel<<<2 * pairs, kThreads, kGemmSmem, st>>>(ta, tb, M, N, K, o, epilogue, status_word());

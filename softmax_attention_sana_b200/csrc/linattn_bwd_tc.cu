@@ -876,18 +876,15 @@ constexpr int kStdNT = 22, kStdNH = 21;
 bool std_split(const RopeDev& r) { return r.n_t == kStdNT && r.n_h == kStdNH && r.n_w == 21; }
 
 void set_bwd_attrs() {
-  static bool done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || done[dev]) return;
-  const int q = (int)(kSmemPerBlock - sizeof(BwdQCtl)), k = (int)kBwdKSmem;
-  cudaFuncSetAttribute(linattn_bwd_q_kernel<true, kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
-  cudaFuncSetAttribute(linattn_bwd_q_kernel<false, kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
-  cudaFuncSetAttribute(linattn_bwd_q_kernel<true, -1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
-  cudaFuncSetAttribute(linattn_bwd_q_kernel<false, -1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
-  cudaFuncSetAttribute(linattn_bwd_k_kernel<kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, k);
-  cudaFuncSetAttribute(linattn_bwd_k_kernel<-1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, k);
-  done[dev] = true;
+  once_per_context(kAttrLinattnBwd, [] {
+    const int q = (int)(kSmemPerBlock - sizeof(BwdQCtl)), k = (int)kBwdKSmem;
+    cudaFuncSetAttribute(linattn_bwd_q_kernel<true, kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
+    cudaFuncSetAttribute(linattn_bwd_q_kernel<false, kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
+    cudaFuncSetAttribute(linattn_bwd_q_kernel<true, -1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
+    cudaFuncSetAttribute(linattn_bwd_q_kernel<false, -1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, q);
+    cudaFuncSetAttribute(linattn_bwd_k_kernel<kStdNT, kStdNH>, cudaFuncAttributeMaxDynamicSharedMemorySize, k);
+    cudaFuncSetAttribute(linattn_bwd_k_kernel<-1, -1>, cudaFuncAttributeMaxDynamicSharedMemorySize, k);
+  });
 }
 
 }  // namespace

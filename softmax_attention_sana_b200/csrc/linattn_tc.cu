@@ -686,17 +686,14 @@ void smem_attr(K kernel, size_t bytes) {
 }
 
 void set_smem_attrs() {
-  static bool done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || done[dev]) return;
-  smem_attr(linattn_state_kernel<kStdNT, kStdNH>, kStateSmem + kRopeSmemMax);
-  smem_attr(linattn_state_kernel<-1, -1>, kStateSmem + kRopeSmemMax);
-  smem_attr(linattn_out_kernel<true, kStdNT, kStdNH>, kOutSmem + kRopeSmemMax);
-  smem_attr(linattn_out_kernel<false, kStdNT, kStdNH>, kOutSmem + kRopeSmemMax);
-  smem_attr(linattn_out_kernel<true, -1, -1>, kOutSmem + kRopeSmemMax);
-  smem_attr(linattn_out_kernel<false, -1, -1>, kOutSmem + kRopeSmemMax);
-  done[dev] = true;
+  once_per_context(kAttrLinattn, [] {
+    smem_attr(linattn_state_kernel<kStdNT, kStdNH>, kStateSmem + kRopeSmemMax);
+    smem_attr(linattn_state_kernel<-1, -1>, kStateSmem + kRopeSmemMax);
+    smem_attr(linattn_out_kernel<true, kStdNT, kStdNH>, kOutSmem + kRopeSmemMax);
+    smem_attr(linattn_out_kernel<false, kStdNT, kStdNH>, kOutSmem + kRopeSmemMax);
+    smem_attr(linattn_out_kernel<true, -1, -1>, kOutSmem + kRopeSmemMax);
+    smem_attr(linattn_out_kernel<false, -1, -1>, kOutSmem + kRopeSmemMax);
+  });
 }
 
 }  // namespace

@@ -432,14 +432,10 @@ sana_status mx_gemm_launch(long long M, int N, int K, const void* xq, const void
       !make_tmap_2d_typed(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wq, (uint64_t)K, (uint64_t)N,
                           (uint64_t)K / 2, BK, BN))
     return fail(SANA_ERR_CUDA, "mx gemm: cuTensorMapEncodeTiled failed");
-  static bool attr[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr[dev]) {
+  once_per_context(BN == 256 ? kAttrMx256 : kAttrMx128, [] {
     cudaFuncSetAttribute(mx_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)MxCfg<BN>::kSmem);
-    attr[dev] = true;
-  }
+  });
   const long long tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < kNumSMs ? tiles : kNumSMs);
   mx_gemm_kernel<BN><<<grid, MxCfg<BN>::kThreads, MxCfg<BN>::kSmem, st>>>(

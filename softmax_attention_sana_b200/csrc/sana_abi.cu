@@ -62,6 +62,18 @@ unsigned long long current_context_id() {
   return id;
 }
 
+void once_per_context(int key, void (*set)()) {
+  static unsigned long long done[kAttrKeys][64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  const bool have_dev = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64;
+  std::lock_guard<std::mutex> lock(mu);
+  const unsigned long long ctx = current_context_id();
+  if (have_dev && ctx != 0 && done[key][dev] == ctx) return;
+  set();
+  if (have_dev) done[key][dev] = current_context_id();
+}
+
 int* status_word() {
   // One slot per device, valid for the context it was looked up in: a device
   // reset gives the device a new context whose copy of the word may sit at a

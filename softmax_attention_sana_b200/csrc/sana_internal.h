@@ -22,6 +22,15 @@ sana_status check_launch(const char* what);
 // Unique id of the calling thread's current CUDA context (cuCtxGetId), 0 if
 // there is none yet or the driver does not provide it.
 unsigned long long current_context_id();
+// Function attributes (the dynamic shared-memory opt-in) belong to a CUDA
+// context: once_per_context runs `set` for a kernel family the first time a
+// call reaches it on a device in a given context (again after a device reset
+// gives the device a new context), under a lock, so no launch of that family
+// runs before its attributes are set.
+enum AttrKey : int {
+  kAttrLinattn = 0, kAttrLinattnBwd, kAttrAnchor, kAttrGemm, kAttrMx128, kAttrMx256, kAttrKeys
+};
+void once_per_context(int key, void (*set)());
 // Device address of the status word of the current device.
 int* status_word();
 
